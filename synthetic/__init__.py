@@ -1,0 +1,151 @@
+"""Seeded synthetic workloads for the SPTS prefill path.
+
+This module only draws random inputs (and the positions of the synthetic
+"salient" keys); it holds none of the method's arithmetic.  The tests, the
+bench and the smoke check take their inputs from here and hand the same
+arrays to the CUDA library and to the CPU oracle.
+
+The real workloads of the method -- LongBench prompts through a trained
+LLaMA-3.1-8B-Instruct -- are not available offline, so these stand in for
+them: a Llama-3.1-8B-shaped layer (32 query / 8 KV heads of 128, hidden 4096,
+SwiGLU 14336) with random N(0, 0.02) weights, N(0, 1) hidden states, and a
+small fraction of keys made salient.  Every draw is from a CPU
+``torch.Generator`` so the values are identical on every machine.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+from fractions import Fraction
+
+import torch
+
+__all__ = ["Workload", "WORKLOADS", "keep_rows", "salient_rows", "make_qkv_f32",
+           "make_hidden", "make_layer_weights", "FUSE_NONE", "FUSE_MAXNORM_ADD", "FUSE_MULTIPLY"]
+
+FUSE_NONE, FUSE_MAXNORM_ADD, FUSE_MULTIPLY = 0, 1, 2
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    N: int
+    Hq: int
+    Hkv: int
+    d: int
+    P: int
+    keep: str                 # keep ratio as an exact decimal string
+    dtype: str = "bf16"       # "f32": Q/K/V given directly; "bf16": a full layer
+    D: int = 0                # hidden size (Hq * d for the Llama shape)
+    F: int = 0                # FFN hidden size (0: attention-only layer)
+    r: int = 0                # LTP rank
+    salient_frac: str = "0"
+    salient_shift: float = 0.0
+    fuse: int = FUSE_MAXNORM_ADD
+    layers: int = 1
+    ratios: tuple = ()
+    seed: int = 1000
+
+    @property
+    def k(self) -> int:
+        return keep_rows(self.keep, self.N)
+
+
+def keep_rows(ratio, n) -> int:
+    """floor(ratio * n) in exact arithmetic."""
+    r = Fraction(str(ratio))
+    return (r.numerator * int(n)) // r.denominator
+
+
+WORKLOADS = {
+    # PAP + select + reduced attention on given fp32 Q/K/V (MHA).
+    "tiny_f32": Workload("tiny_f32", N=512, Hq=4, Hkv=4, d=64, P=16, keep="0.25", dtype="f32",
+                         salient_frac="0.02", salient_shift=3.0, seed=1001),
+    # Llama-3.1-8B-shaped attention-only layer at 8K tokens.
+    "attn_8k": Workload("attn_8k", N=8192, Hq=32, Hkv=8, d=128, P=64, keep="0.4", D=4096,
+                        salient_frac="0.02", salient_shift=3.0, seed=1002),
+    # Full SPTS layer (PAP + LTP) at 32K and 128K tokens.
+    "layer_32k": Workload("layer_32k", N=32768, Hq=32, Hkv=8, d=128, P=64, keep="0.3", D=4096,
+                          F=14336, r=256, salient_frac="0.02", salient_shift=3.0, seed=1003),
+    "layer_128k": Workload("layer_128k", N=131072, Hq=32, Hkv=8, d=128, P=128, keep="0.2", D=4096,
+                           F=14336, r=256, salient_frac="0.01", salient_shift=4.0, seed=1004),
+    # MSDP: 8 layers in 4 stages of 2, candidate ratios 0.8/0.6/0.4/0.25.
+    "msdp_32k": Workload("msdp_32k", N=32768, Hq=32, Hkv=8, d=128, P=64, keep="0.8", D=4096,
+                         F=14336, r=256, layers=8, ratios=("0.8", "0.6", "0.4", "0.25"), seed=1005),
+    # Small shapes for full element-by-element parity (ragged N, several tiles).
+    "layer_small": Workload("layer_small", N=1000, Hq=8, Hkv=2, d=128, P=16, keep="0.3", D=1024,
+                            F=1536, r=64, salient_frac="0.02", salient_shift=3.0, seed=1101),
+    "msdp_small": Workload("msdp_small", N=600, Hq=8, Hkv=2, d=128, P=16, keep="0.8", D=1024,
+                           F=1024, r=64, layers=8, ratios=("0.8", "0.6", "0.4", "0.25"), seed=1102),
+}
+
+
+def _gen(seed):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def salient_rows(n, p, frac, seed):
+    """floor(frac * n) distinct rows drawn from [0, n - p), sorted."""
+    count = keep_rows(frac, n)
+    if count == 0:
+        return torch.zeros(0, dtype=torch.int32)
+    g = _gen(seed + 7)
+    perm = torch.randperm(n - p, generator=g)[:count]
+    return torch.sort(perm).values.to(torch.int32)
+
+
+def make_qkv_f32(wl: Workload):
+    """fp32 Q, K, V [N, H, d] ~ N(0, 1) with salient keys (the tiny MHA case).
+
+    Salience: for each head, the keys at ``salient_rows`` get
+    shift * unit(mean of that head's probe queries), the probes being the last
+    P rows.  Returns (q, k, v, pos int32, salient rows).
+    """
+    g = _gen(wl.seed)
+    q = torch.randn(wl.N, wl.Hq, wl.d, generator=g, dtype=torch.float32)
+    k = torch.randn(wl.N, wl.Hkv, wl.d, generator=g, dtype=torch.float32)
+    v = torch.randn(wl.N, wl.Hkv, wl.d, generator=g, dtype=torch.float32)
+    rows = salient_rows(wl.N, wl.P, wl.salient_frac, wl.seed)
+    if len(rows):
+        G = wl.Hq // wl.Hkv
+        for gidx in range(wl.Hkv):
+            mean = q[wl.N - wl.P:, gidx * G:(gidx + 1) * G, :].reshape(-1, wl.d).double().mean(0)
+            u = (mean / mean.norm()).float()
+            k[rows.long(), gidx, :] += wl.salient_shift * u
+    pos = torch.arange(wl.N, dtype=torch.int32)
+    return q, k, v, pos, rows
+
+
+def make_hidden(wl: Workload, n=None):
+    """Residual-stream input h [n, D]: N(0, 1) values rounded to bf16, held in fp32."""
+    n = wl.N if n is None else n
+    g = _gen(wl.seed)
+    return torch.randn(n, wl.D, generator=g, dtype=torch.float32).to(torch.bfloat16).float()
+
+
+def make_layer_weights(wl: Workload, layer: int = 0):
+    """bf16 weights of one Llama-shaped layer, nn.Linear layout, ~N(0, 0.02).
+
+    Keys: w_q [Hq*d, D], w_k / w_v [Hkv*d, D], w_o [D, Hq*d]; when F > 0 also
+    w_gate / w_up [F, D], w_down [D, F], ltp_a [r, D], ltp_b [D, r].  Norm
+    weights are ones.
+    """
+    g = _gen(wl.seed * 1000 + 17 + 101 * layer)
+    D, hd, kd = wl.D, wl.Hq * wl.d, wl.Hkv * wl.d
+
+    def w(o, i):
+        return (0.02 * torch.randn(o, i, generator=g, dtype=torch.float32)).to(torch.bfloat16)
+
+    out = dict(w_q=w(hd, D), w_k=w(kd, D), w_v=w(kd, D), w_o=w(D, hd))
+    if wl.F:
+        out.update(w_gate=w(wl.F, D), w_up=w(wl.F, D), w_down=w(D, wl.F),
+                   ltp_a=w(wl.r, D), ltp_b=w(D, wl.r))
+    out["norm_attn"] = torch.ones(D, dtype=torch.bfloat16)
+    out["norm_ffn"] = torch.ones(D, dtype=torch.bfloat16)
+    return out
+
+
+def with_overrides(wl: Workload, **kw) -> Workload:
+    return replace(wl, **kw)
