@@ -1,0 +1,103 @@
+"""GPU parity of the bf16 tensor-core kernels (tcgen05) against the oracle:
+PAP probe scores, the LTP score, reduced GQA attention and one full layer."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tests.gpu_util import assert_bf16_close, assert_close, band_check, np64
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import token_skipping_sparse_b200 as S
+
+rng = np.random.default_rng(11)
+
+
+def _positions(n, span_factor=3):
+    return np.sort(rng.choice(n * span_factor, n, replace=False)).astype(np.int32)
+
+
+@pytest.mark.parametrize("Nc,k,Hq,Hkv", [(1000, 300, 8, 2), (513, 200, 4, 4), (1000, 250, 8, 4),
+                                         (1000, 300, 16, 2), (5000, 1500, 32, 8), (129, 1, 8, 2), (128, 128, 8, 2)])
+def test_reduced_attention_bf16(Nc, k, Hq, Hkv):
+    pos = _positions(Nc)
+    sel = np.sort(rng.choice(Nc, k, replace=False))
+    q = torch.randn(k, Hq, 128).to(torch.bfloat16)
+    kk = torch.randn(Nc, Hkv, 128).to(torch.bfloat16)
+    v = torch.randn(Nc, Hkv, 128).to(torch.bfloat16)
+    o = S.spts_reduced_attention(q.cuda(), torch.from_numpy(pos[sel]).cuda(), kk.cuda(), v.cuda(),
+                                 torch.from_numpy(pos).cuda())
+    want = O.reduced_attention(np64(q), pos[sel], np64(kk), np64(v), pos)
+    got = np64(o)
+    assert_close(got, want, 2e-2, "reduced attention bf16")
+    assert np.mean(np.abs(got - want)) < 2e-3
+
+
+@pytest.mark.parametrize("Nc,P,Hq,Hkv", [(1000, 16, 8, 2), (3000, 64, 32, 8), (2000, 128, 32, 8), (300, 64, 8, 8),
+                                         (700, 20, 8, 4)])
+def test_probe_scores_bf16(Nc, P, Hq, Hkv):
+    pos = _positions(Nc)
+    q = torch.randn(P, Hq, 128).to(torch.bfloat16)
+    kk = torch.randn(Nc, Hkv, 128).to(torch.bfloat16)
+    s, g = S.spts_probe_scores(q.cuda(), torch.from_numpy(pos[-P:]).cuda(), kk.cuda(), torch.from_numpy(pos).cuda(),
+                               group_scores=True)
+    ws_, wg = O.probe_scores(np64(q), pos[-P:], np64(kk), pos)
+    tol = 1e-3 * ws_.max() + 1e-5
+    assert_close(s.cpu().numpy(), ws_, tol, "probe scores")
+    assert_close(g.cpu().numpy(), wg, tol, "group scores")
+    assert abs(float(s.double().sum()) - P * Hq) < 1e-3 * P * Hq
+
+
+@pytest.mark.parametrize("Nc,D,r,Dout", [(1000, 1024, 64, 1024), (300, 4096, 256, 4096), (129, 512, 128, 768)])
+def test_ltp_scores_bf16(Nc, D, r, Dout):
+    x = torch.randn(Nc, D).to(torch.bfloat16)
+    A = (0.02 * torch.randn(r, D)).to(torch.bfloat16)
+    B = (0.02 * torch.randn(Dout, r)).to(torch.bfloat16)
+    c = S.spts_ltp_scores(x.cuda(), A.cuda(), B.cuda())
+    want = O.ltp_scores(np64(x), np64(A), np64(B))
+    assert_close(c.cpu().numpy(), want, 1e-3 * want.max(), "ltp scores")
+
+
+def _layer_case(name):
+    from synthetic import WORKLOADS, make_hidden, make_layer_weights, salient_rows
+    wl = WORKLOADS[name]
+    h = make_hidden(wl)
+    W = make_layer_weights(wl)
+    sal = salient_rows(wl.N, wl.P, wl.salient_frac, wl.seed)
+    pos = torch.arange(wl.N, dtype=torch.int32)
+    return wl, h, W, sal, pos
+
+
+def test_layer_small_matches_oracle():
+    wl, h, W, sal, pos = _layer_case("layer_small")
+    Wd = {n: t.cuda() for n, t in W.items()}
+    desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k, fuse=wl.fuse,
+                        salient_rows=sal.cuda(), salient_shift=wl.salient_shift)
+    hd = h.cuda()
+    out = S.spts_layer_forward(hd, pos.cuda(), desc, Wd, outputs=True)
+    S.check_device_status()
+    ow = O.LayerWeights(**{n: np64(t) for n, t in W.items()})
+    cfg = O.LayerConfig(Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, P=wl.P, k=wl.k, fuse=wl.fuse,
+                        salient_rows=sal.numpy(), salient_shift=wl.salient_shift)
+    tr = {}
+    O.layer_forward(np64(h), pos.numpy(), ow, cfg, tr)
+    s = out["s"].cpu().numpy()
+    assert_close(s, tr["s"], 1e-3 * tr["s"].max(), "probe scores")
+    ia = out["idx_attn"].cpu().numpy()
+    band_check(ia, tr["idx_attn"], tr["s"], tr["tau_attn"])
+    # reduced attention rows: oracle computes every row, compare at the GPU's picks
+    q_all = O.bf16_round(O.rope((tr["xn"] @ ow.w_q.T).reshape(wl.N, wl.Hq, wl.d), pos.numpy()))
+    o_all = O.bf16_round(O.reduced_attention(q_all, pos.numpy(), tr["k"], tr["v"], pos.numpy()))
+    assert_bf16_close(np64(out["o_sel"]), o_all[ia], 2e-2, "o_sel")
+    same = np.array_equal(ia, tr["idx_attn"])
+    if same:
+        assert_close(np64(out["h_attn"]), tr["h_attn"], 2e-2, "h after attention")
+        c = out["c"].cpu().numpy()
+        assert_close(c, tr["c"], 1e-3 * tr["c"].max(), "ltp scores")
+        idf = out["idx_ffn"].cpu().numpy()
+        band_check(idf, tr["idx_ffn"], tr["f"], tr["tau_ffn"])
+        if np.array_equal(idf, tr["idx_ffn"]):
+            assert_close(np64(hd), tr["h_out"], 2e-2, "h out")

@@ -1,0 +1,337 @@
+// gemm.cu -- bf16 tensor-core GEMM acc = A W^T on sm_100a with fused epilogues.
+//
+// This is the projection engine of the SPTS layer: K/V (+RoPE) for every
+// candidate, Q for the probe rows and for the selected rows, the O
+// projection added into the residual at the selected rows, and the reduced
+// SwiGLU FFN (gate/up with the SwiGLU product, down added into the residual).
+//
+// Design (one CTA per SM, persistent over 128 x 256 output tiles):
+//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 per stage into
+//               a 4-stage ring of 128-byte-swizzled shared memory;
+//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
+//               K=16) into one of two TMEM accumulators (2 x 256 columns);
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (warp w reads
+//               TMEM lanes 32*(w%4)..+31), then the fused epilogue and the
+//               global stores, overlapping the next tile's main loop.
+// Tiles are visited in groups of 16 M-tiles (M fastest inside a group) so a
+// wave of 148 CTAs shares both operands through L2.
+// Every barrier wait is bounded (see sm100.cuh).
+#include "host.hpp"
+#include "rowops.cuh"
+#include "sm100.cuh"
+
+namespace spts {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
+constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 48 KB
+constexpr int GROUP_M = 16;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+
+struct Params {
+  int M, N, K;         // N: output columns of W (for SWIGLU: of W_gate and of W_up each)
+  int tiles_m, tiles_n;
+  void *out;
+  const int32_t *rows;
+  const int32_t *row_pos;
+  uint32_t *status;
+  uint64_t wait_ns;
+  RopeFreqs freqs;
+};
+
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int &tm, int &tn) {
+  const int per_group = GROUP_M * tiles_n;
+  const int grp = t / per_group;
+  const int first_m = grp * GROUP_M;
+  const int gm = min(GROUP_M, tiles_m - first_m);
+  const int r = t - grp * per_group;
+  tm = first_m + r % gm;
+  tn = r / gm;
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float *v) {
+  uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 o;
+    o.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    o.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    o.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    o.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d4[q] = o;
+  }
+}
+
+__device__ __forceinline__ void rope_angle_f(int32_t pos, double inv_freq, float *c, float *s) {
+  const double two_pi = 6.283185307179586476925286766559;
+  double a = static_cast<double>(pos) * inv_freq;
+  a -= two_pi * rint(a / two_pi);
+  sincosf(static_cast<float>(a), s, c);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * A_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  uint64_t *full = bars, *empty = bars + STAGES, *tfull = bars + 2 * STAGES, *tempty = tfull + 2,
+           *drain = tempty + 2;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int kblocks = p.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      if (EPI == SPTS_EPI_SWIGLU) tma_prefetch_desc(&tmB2);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+        int tm, tn;
+        tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+        const int m0 = tm * BM;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, p.wait_ns, 0x11u)) break;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          uint8_t *a_dst = sA + stage * A_BYTES;
+          uint8_t *b_dst = sB + stage * B_BYTES;
+          tma_load_2d(a_dst, &tmA, &full[stage], kb * BK, m0);
+          if (EPI == SPTS_EPI_SWIGLU) {
+            tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, tn * 128);
+            tma_load_2d(b_dst + B_BYTES / 2, &tmB2, &full[stage], kb * BK, tn * 128);
+          } else {
+            tma_load_2d(b_dst, &tmB, &full[stage], kb * BK, tn * BN);
+            tma_load_2d(b_dst + B_BYTES / 2, &tmB, &full[stage], kb * BK, tn * BN + 128);
+          }
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag) {
+        // let the copies already in flight land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s)) mbar_drain(&full[s], (issued_phase >> s) & 1u, p.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, p.wait_ns, 0x12u)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, p.wait_ns, 0x13u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = sdesc_k_sw128(smem_u32(sA + stage * A_BYTES));
+          const uint64_t bdesc = sdesc_k_sw128(smem_u32(sB + stage * B_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+          tc_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) tc_commit(&tfull[acc]);
+      }
+      // every MMA issued so far must finish before TMEM is released
+      tc_commit(drain);
+      mbar_drain(drain, 0, p.status);
+    }
+    __syncwarp();
+  } else {
+    // epilogue warps 2..5 -> TMEM lane quadrant warp % 4
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    int local = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, p.wait_ns, 0x14u);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      int tm, tn;
+      tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+      const int64_t row = static_cast<int64_t>(tm) * BM + row_in_tile;
+      const bool live = row < p.M;
+      const uint32_t tbase = tmem_addr(tmem_base, quad * 32, acc * BN);
+      if (EPI == SPTS_EPI_STORE) {
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c * 32, r);
+          tmem_ld_wait();
+          if (live) store_bf16x32(out + row * p.N + tn * BN + c * 32, reinterpret_cast<float *>(r));
+        }
+      } else if (EPI == SPTS_EPI_ROPE) {
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
+        const int32_t pos = live ? p.row_pos[row] : 0;
+#pragma unroll 1
+        for (int hc = 0; hc < BN / 128; ++hc) {     // heads of 128 columns in this tile
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {             // pairs i in [32c, 32c+32), partner i+64
+            uint32_t lo[32], hi[32];
+            tmem_ld32(tbase + hc * 128 + c * 32, lo);
+            tmem_ld32(tbase + hc * 128 + 64 + c * 32, hi);
+            tmem_ld_wait();
+            float *xl = reinterpret_cast<float *>(lo);
+            float *xh = reinterpret_cast<float *>(hi);
+            float yl[32], yh[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              float cs, sn;
+              rope_angle_f(pos, p.freqs.inv_freq[c * 32 + i], &cs, &sn);
+              yl[i] = xl[i] * cs - xh[i] * sn;
+              yh[i] = xh[i] * cs + xl[i] * sn;
+            }
+            if (live) {
+              __nv_bfloat16 *o = out + row * p.N + tn * BN + hc * 128;
+              store_bf16x32(o + c * 32, yl);
+              store_bf16x32(o + 64 + c * 32, yh);
+            }
+          }
+        }
+      } else if (EPI == SPTS_EPI_SWIGLU) {
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tbase + c * 32, g);
+          tmem_ld32(tbase + 128 + c * 32, u);
+          tmem_ld_wait();
+          float y[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = silu(__uint_as_float(g[i])) * __uint_as_float(u[i]);
+          if (live) store_bf16x32(out + row * p.N + tn * 128 + c * 32, y);
+        }
+      } else {  // SCATTER_ADD into fp32 rows
+        float *out = static_cast<float *>(p.out);
+        const int64_t orow = live ? p.rows[row] : 0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c * 32, r);
+          tmem_ld_wait();
+          if (live) {
+            float4 *dst = reinterpret_cast<float4 *>(out + orow * p.N + tn * BN + c * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              float4 h = dst[q];
+              h.x += __uint_as_float(r[4 * q + 0]);
+              h.y += __uint_as_float(r[4 * q + 1]);
+              h.z += __uint_as_float(r[4 * q + 2]);
+              h.w += __uint_as_float(r[4 * q + 3]);
+              dst[q] = h;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+template <int EPI>
+spts_status launch_epi(const GemmArgs &g, const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tb2,
+                       Params &p, cudaStream_t s) {
+  SPTS_CUDA_TRY(cudaFuncSetAttribute(gemm_bf16_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(SMEM_BYTES)));
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  gemm_bf16_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, tb2, p);
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+}  // namespace
+
+spts_status launch_gemm(const GemmArgs &g, cudaStream_t s) {
+  if (g.M == 0) return SPTS_OK;
+  CUtensorMap ta, tb, tb2;
+  SPTS_TRY(tmap_bf16_2d(&ta, g.A, static_cast<uint64_t>(g.M), g.K, g.K, 128));
+  SPTS_TRY(tmap_bf16_2d(&tb, g.W, static_cast<uint64_t>(g.N), g.K, g.K, 128));
+  if (g.epi == SPTS_EPI_SWIGLU)
+    SPTS_TRY(tmap_bf16_2d(&tb2, g.W2, static_cast<uint64_t>(g.N), g.K, g.K, 128));
+  else
+    tb2 = tb;
+  Params p{};
+  p.M = static_cast<int>(g.M);
+  p.N = g.N;
+  p.K = g.K;
+  p.tiles_m = static_cast<int>((g.M + BM - 1) / BM);
+  p.tiles_n = g.epi == SPTS_EPI_SWIGLU ? g.N / 128 : g.N / BN;
+  p.out = g.out;
+  p.rows = g.rows;
+  p.row_pos = g.row_pos;
+  p.status = g.status;
+  p.wait_ns = wait_limit_ns();
+  if (g.epi == SPTS_EPI_ROPE) fill_rope_freqs(&p.freqs, 128, g.theta);
+  switch (g.epi) {
+    case SPTS_EPI_STORE: return launch_epi<SPTS_EPI_STORE>(g, ta, tb, tb2, p, s);
+    case SPTS_EPI_ROPE: return launch_epi<SPTS_EPI_ROPE>(g, ta, tb, tb2, p, s);
+    case SPTS_EPI_SWIGLU: return launch_epi<SPTS_EPI_SWIGLU>(g, ta, tb, tb2, p, s);
+    default: return launch_epi<SPTS_EPI_SCATTER_ADD>(g, ta, tb, tb2, p, s);
+  }
+}
+
+}  // namespace spts

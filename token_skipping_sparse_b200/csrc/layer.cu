@@ -1,0 +1,167 @@
+// layer.cu -- one SPTS prefill layer composed from the kernels, in the order
+// of Fig. 2: probe (PAP) -> select -> reduced attention -> O projection into
+// the selected rows -> LTP score -> fuse + select -> reduced FFN.
+#include <cstring>
+
+#include "host.hpp"
+#include "rowops.cuh"
+
+using namespace spts;
+
+namespace {
+
+struct LayerBufs {
+  void *xn, *kk, *vv, *qprobe, *xsel, *qsel, *osel, *act;
+  float *s, *group, *stats, *c, *f;
+  int32_t *idx_a, *idx_f, *qpos;
+};
+
+// Carves the workspace; with cv.base == nullptr it only measures.
+void carve(Carver &cv, const spts_layer_desc *L, int64_t Nc, LayerBufs &b) {
+  const int64_t k = L->k;
+  const size_t D = L->D, hq = static_cast<size_t>(L->Hq) * L->d, hk = static_cast<size_t>(L->Hkv) * L->d;
+  b.xn = cv.take(Nc * D * 2);
+  b.kk = cv.take(Nc * hk * 2);
+  b.vv = cv.take(Nc * hk * 2);
+  b.qprobe = cv.take(static_cast<size_t>(L->P) * hq * 2);
+  b.xsel = cv.take(k * D * 2);
+  b.qsel = cv.take(k * hq * 2);
+  b.osel = cv.take(k * hq * 2);
+  b.act = cv.take(static_cast<size_t>(k) * (L->F > 0 ? L->F : 1) * 2);
+  b.s = static_cast<float *>(cv.take(Nc * 4));
+  b.group = static_cast<float *>(cv.take(static_cast<size_t>(L->Hkv) * Nc * 4));
+  b.stats = static_cast<float *>(cv.take(probe_bf16_stats_bytes(L->P, L->Hq, Nc)));
+  b.c = static_cast<float *>(cv.take(Nc * 4));
+  b.f = static_cast<float *>(cv.take(Nc * 4));
+  b.idx_a = static_cast<int32_t *>(cv.take(k * 4));
+  b.idx_f = static_cast<int32_t *>(cv.take(k * 4));
+  b.qpos = static_cast<int32_t *>(cv.take(k * 4));
+}
+
+spts_status check_layer(const spts_layer_desc *L, const spts_layer_weights *W, int64_t Nc) {
+  const char *who = "spts_layer_forward";
+  SPTS_REQUIRE(L && W, SPTS_ERR_INVALID, "%s: NULL descriptor", who);
+  SPTS_REQUIRE(L->d == 128 && L->Hq > 0 && L->Hkv > 0 && L->Hq % L->Hkv == 0, SPTS_ERR_UNSUPPORTED,
+               "%s: needs d = 128 and Hq %% Hkv == 0", who);
+  const int G = L->Hq / L->Hkv;
+  SPTS_REQUIRE(G == 1 || G == 2 || G == 4 || G == 8, SPTS_ERR_UNSUPPORTED, "%s: Hq/Hkv must be 1, 2, 4 or 8", who);
+  SPTS_REQUIRE(L->D % 256 == 0 && (L->Hq * L->d) % 256 == 0 && (L->Hkv * L->d) % 256 == 0, SPTS_ERR_SHAPE,
+               "%s: D, Hq*d and Hkv*d must be multiples of 256", who);
+  SPTS_REQUIRE(L->P >= 1 && L->P <= 128 && L->P <= L->k && L->k <= Nc && Nc < (int64_t(1) << 31), SPTS_ERR_SHAPE,
+               "%s: need 1 <= P <= 128, P <= k <= Nc", who);
+  SPTS_REQUIRE(W->w_q && W->w_k && W->w_v && W->w_o, SPTS_ERR_INVALID, "%s: attention weights missing", who);
+  if (L->F > 0) {
+    SPTS_REQUIRE(L->F % 128 == 0 && L->r >= 64 && L->r <= 256 && L->r % 64 == 0, SPTS_ERR_SHAPE,
+                 "%s: need F %% 128 == 0 and r in {64,...,256} step 64", who);
+    SPTS_REQUIRE(W->w_gate && W->w_up && W->w_down && W->ltp_a && W->ltp_b, SPTS_ERR_INVALID,
+                 "%s: FFN / LTP weights missing", who);
+    SPTS_REQUIRE(L->fuse >= SPTS_FUSE_NONE && L->fuse <= SPTS_FUSE_MULTIPLY, SPTS_ERR_INVALID, "%s: bad fusion",
+                 who);
+  }
+  SPTS_REQUIRE(L->n_salient == 0 || L->salient_rows != nullptr, SPTS_ERR_INVALID, "%s: salient rows NULL", who);
+  return SPTS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t spts_layer_forward_workspace(const spts_layer_desc *L, int64_t Nc) {
+  if (L == nullptr || Nc <= 0) return kStatusBytes;
+  Carver cv(nullptr, 0);
+  LayerBufs b;
+  carve(cv, L, Nc, b);
+  return cv.off;
+}
+
+spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weights *W, float *h, const int32_t *pos,
+                               int64_t Nc, const spts_layer_outputs *out, void *ws, size_t ws_bytes,
+                               spts_stream stream) {
+  SPTS_TRY(check_layer(L, W, Nc));
+  SPTS_REQUIRE(h && pos && aligned(h, 16) && aligned(pos, 4), SPTS_ERR_INVALID, "spts_layer_forward: bad h/pos");
+  SPTS_TRY(check_ws(ws, ws_bytes, spts_layer_forward_workspace(L, Nc), "spts_layer_forward"));
+  spts_layer_outputs none;
+  memset(&none, 0, sizeof(none));
+  const spts_layer_outputs &o = out ? *out : none;
+  Carver cv(ws, ws_bytes);
+  LayerBufs b;
+  carve(cv, L, Nc, b);
+  uint32_t *st = cv.status();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int D = L->D, P = L->P, hq = L->Hq * L->d, hk = L->Hkv * L->d;
+  const int64_t k = L->k;
+  float *sc = o.s ? o.s : b.s;
+  int32_t *idx_a = o.idx_attn ? o.idx_attn : b.idx_a;
+  void *osel = o.o_sel ? o.o_sel : b.osel;
+  const float scale = 1.0f / sqrtf(static_cast<float>(L->d));
+  auto mark = [&](int i) -> spts_status {
+    if (o.stage_events != nullptr) {
+      SPTS_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(o.stage_events[i]), s));
+    }
+    return SPTS_OK;
+  };
+
+  // a1-a2: norm, K (+RoPE) / V for every candidate, Q (+RoPE) for the probe rows
+  SPTS_TRY(mark(0));
+  SPTS_TRY(launch_rmsnorm_rows(h, nullptr, Nc, D, W->norm_attn, L->eps, b.xn, s));
+  SPTS_TRY(mark(1));
+  GemmArgs gk{b.xn, Nc, D, W->w_k, nullptr, hk, SPTS_EPI_ROPE, b.kk, nullptr, pos, L->theta, st};
+  SPTS_TRY(launch_gemm(gk, s));
+  SPTS_TRY(mark(2));
+  GemmArgs gv{b.xn, Nc, D, W->w_v, nullptr, hk, SPTS_EPI_STORE, b.vv, nullptr, nullptr, 0.0, st};
+  SPTS_TRY(launch_gemm(gv, s));
+  SPTS_TRY(mark(3));
+  const void *xtail = static_cast<const char *>(b.xn) + static_cast<size_t>(Nc - P) * D * 2;
+  GemmArgs gq{xtail, P, D, W->w_q, nullptr, hq, SPTS_EPI_ROPE, b.qprobe, nullptr, pos + (Nc - P), L->theta, st};
+  SPTS_TRY(launch_gemm(gq, s));
+  if (L->n_salient > 0)
+    SPTS_TRY(launch_inject_salience(b.kk, Nc, b.qprobe, P, L->Hq, L->Hkv, L->d, L->salient_rows, L->n_salient,
+                                    L->salient_shift, st, s));
+  SPTS_TRY(mark(4));
+
+  // a3-a4: probe scores, MHA selection
+  SPTS_TRY(launch_probe_bf16(b.qprobe, pos + (Nc - P), P, b.kk, pos, Nc, L->Hq, L->Hkv, scale, b.group, b.stats, st,
+                             s));
+  SPTS_TRY(launch_sum_groups(b.group, L->Hkv, Nc, sc, s));
+  SPTS_TRY(mark(5));
+  SPTS_TRY(launch_select_topk(sc, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, Nc, k, P, idx_a, nullptr, nullptr, st, s));
+  SPTS_TRY(mark(6));
+
+  // a5-a7: Q for the selected rows, reduced attention, O projection into h
+  SPTS_TRY(launch_gather_i32(pos, idx_a, k, b.qpos, s));
+  SPTS_TRY(launch_gather_rows(b.xn, Nc, idx_a, k, static_cast<int64_t>(D) * 2, b.xsel, nullptr, nullptr, st, s));
+  SPTS_TRY(mark(7));
+  GemmArgs gqs{b.xsel, k, D, W->w_q, nullptr, hq, SPTS_EPI_ROPE, b.qsel, nullptr, b.qpos, L->theta, st};
+  SPTS_TRY(launch_gemm(gqs, s));
+  SPTS_TRY(mark(8));
+  SPTS_TRY(launch_attention_bf16(b.qsel, b.qpos, k, b.kk, b.vv, pos, Nc, L->Hq, L->Hkv, scale, osel, st, s));
+  SPTS_TRY(mark(9));
+  GemmArgs go{osel, k, hq, W->w_o, nullptr, D, SPTS_EPI_SCATTER_ADD, h, idx_a, nullptr, 0.0, st};
+  SPTS_TRY(launch_gemm(go, s));
+  if (o.h_attn) SPTS_CUDA_TRY(cudaMemcpyAsync(o.h_attn, h, static_cast<size_t>(Nc) * D * 4, cudaMemcpyDeviceToDevice, s));
+  SPTS_TRY(mark(10));
+  if (L->F <= 0) {
+    for (int i = 11; i < SPTS_LAYER_STAGE_EVENTS; ++i) SPTS_TRY(mark(i));
+    return SPTS_OK;
+  }
+
+  // a8-a10: LTP score, fused FFN selection, reduced FFN
+  float *c = o.c ? o.c : b.c;
+  float *f = o.f ? o.f : b.f;
+  int32_t *idx_f = o.idx_ffn ? o.idx_ffn : b.idx_f;
+  SPTS_TRY(launch_rmsnorm_rows(h, nullptr, Nc, D, W->norm_ffn, L->eps, b.xn, s));
+  SPTS_TRY(mark(11));
+  SPTS_TRY(launch_ltp_bf16(b.xn, Nc, D, W->ltp_a, L->r, W->ltp_b, D, c, st, s));
+  SPTS_TRY(mark(12));
+  SPTS_TRY(launch_select_topk(sc, c, L->fuse, L->w_a, L->w_b, Nc, k, P, idx_f, f, nullptr, st, s));
+  SPTS_TRY(launch_gather_rows(b.xn, Nc, idx_f, k, static_cast<int64_t>(D) * 2, b.xsel, nullptr, nullptr, st, s));
+  SPTS_TRY(mark(13));
+  GemmArgs g1{b.xsel, k, D, W->w_gate, W->w_up, L->F, SPTS_EPI_SWIGLU, b.act, nullptr, nullptr, 0.0, st};
+  SPTS_TRY(launch_gemm(g1, s));
+  SPTS_TRY(mark(14));
+  GemmArgs g2{b.act, k, L->F, W->w_down, nullptr, D, SPTS_EPI_SCATTER_ADD, h, idx_f, nullptr, 0.0, st};
+  SPTS_TRY(launch_gemm(g2, s));
+  return mark(15);
+}
+
+}  // extern "C"

@@ -1,0 +1,232 @@
+// ltp.cu -- Low-rank Transformation Probing score on sm_100a (Fig. 2(b),
+// Table 6, Table A): c_i = || (x_i A^T) B^T ||_2.
+//
+// One CTA per tile of 128 rows, a chained pair of tcgen05 GEMMs that never
+// writes the proxy output to memory:
+//   phase 1  T = X A^T   (M=128, N=r, K=D) accumulated in TMEM, then read
+//            back, rounded to bf16 and stored in shared memory in the UMMA
+//            K-major swizzled layout, where it becomes the A operand of
+//   phase 2  Y = T B^T   (M=128, N=256 per chunk, K=r), chunk by chunk over
+//            the Dout outputs into two ping-pong TMEM accumulators; the
+//            epilogue warps fold every chunk into a per-row sum of squares.
+// Per row only 2*D bytes of X are read from HBM; A and B (2 x r x D bf16)
+// are shared by all CTAs through L2.  Waits are bounded.
+#include "host.hpp"
+#include "rowops.cuh"
+#include "sm100.cuh"
+
+namespace spts {
+namespace {
+
+constexpr int THREADS = 192;
+constexpr int STAGES = 3;
+constexpr int SLOT = 48 * 1024;
+constexpr int X_BYTES = 128 * 64 * 2;  // 16 KB
+constexpr int CHUNK_BYTES = 128 * 64 * 2;
+constexpr int OFF_TS = STAGES * SLOT;               // T in bf16: r/64 chunks of 16 KB
+constexpr int OFF_BAR = OFF_TS + 4 * CHUNK_BYTES;
+constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 256;
+
+struct Params {
+  int M, D, r, Dout;
+  float *scores;
+  uint32_t *status;
+  uint64_t wait_ns;
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+    ltp_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
+               const __grid_constant__ CUtensorMap tmB, const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sT = smem + OFF_TS;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint64_t *full = bars, *empty = bars + STAGES, *t_full = bars + 2 * STAGES, *ts_ready = t_full + 1,
+           *acc_full = ts_ready + 1, *acc_empty = acc_full + 2, *drain = acc_empty + 2;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128;
+  const int kb1 = p.D / 64, kb2 = p.r / 64, nch = p.Dout / 256;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(t_full, 1);
+    mbar_init(ts_ready, 128);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      uint32_t issued = 0, par = 0;
+      const int total = kb1 + nch * kb2;
+      for (int i = 0; i < total; ++i) {
+        const int st = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status, p.wait_ns, 0x51u)) break;
+        uint8_t *slot = smem + st * SLOT;
+        if (i < kb1) {
+          mbar_arrive_expect_tx(&full[st], X_BYTES + p.r * 128);
+          tma_load_2d(slot, &tmX, &full[st], i * 64, m0);
+          tma_load_2d(slot + X_BYTES, &tmA, &full[st], i * 64, 0);
+        } else {
+          const int j = i - kb1;
+          mbar_arrive_expect_tx(&full[st], 256 * 128);
+          tma_load_2d(slot, &tmB, &full[st], (j % kb2) * 64, (j / kb2) * 256);
+        }
+        issued |= 1u << st;
+        par = (par & ~(1u << st)) | (ph << st);
+      }
+      if (*abort_flag)
+        for (int st = 0; st < STAGES; ++st)
+          if (issued & (1u << st)) mbar_drain(&full[st], (par >> st) & 1u, p.status);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc1 = idesc_bf16_f32(128, p.r, 0, 0);
+      constexpr uint32_t idesc2 = idesc_bf16_f32(128, 256, 0, 0);
+      bool ok = true;
+      int i = 0;
+      for (int kb = 0; ok && kb < kb1; ++kb, ++i) {
+        const int st = i % STAGES;
+        if (!mbar_wait(&full[st], (i / STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x52u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t base = smem_u32(smem + st * SLOT);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tmem, sdesc_k_sw128(base) + 2 * kk, sdesc_k_sw128(base + X_BYTES) + 2 * kk, idesc1,
+                      (kb | kk) != 0);
+        tc_commit(&empty[st]);
+      }
+      if (ok) tc_commit(t_full);
+      if (ok) ok = mbar_wait(ts_ready, 0, abort_flag, p.status, p.wait_ns, 0x53u);
+      tc_fence_after();
+      const uint32_t t_addr = smem_u32(sT);
+      for (int nc = 0; ok && nc < nch; ++nc) {
+        const int acc = nc & 1;
+        if (!mbar_wait(&acc_empty[acc], ((nc >> 1) & 1) ^ 1u, abort_flag, p.status, p.wait_ns, 0x54u)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < kb2; ++kb, ++i) {
+          const int st = i % STAGES;
+          if (!mbar_wait(&full[st], (i / STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x55u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t base = smem_u32(smem + st * SLOT);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tmem + acc * 256, sdesc_k_sw128(t_addr + kb * CHUNK_BYTES) + 2 * kk,
+                        sdesc_k_sw128(base) + 2 * kk, idesc2, (kb | kk) != 0);
+          tc_commit(&empty[st]);
+        }
+        if (ok) tc_commit(&acc_full[acc]);
+      }
+      tc_commit(drain);
+      mbar_drain(drain, 0, p.status);
+    }
+    __syncwarp();
+  } else {
+    const int quad = warp & 3;
+    const int rr = quad * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    bool ok = mbar_wait(t_full, 0, abort_flag, p.status, p.wait_ns, 0x56u);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      // T row -> bf16 -> shared memory (K-major, 128-byte swizzle)
+      for (int c0 = 0; c0 < p.r; c0 += 32) {
+        uint32_t t[32];
+        tmem_ld32(lane_base + c0, t);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(t[8 * q + 0]), __uint_as_float(t[8 * q + 1]));
+          v.y = pack_bf16x2(__uint_as_float(t[8 * q + 2]), __uint_as_float(t[8 * q + 3]));
+          v.z = pack_bf16x2(__uint_as_float(t[8 * q + 4]), __uint_as_float(t[8 * q + 5]));
+          v.w = pack_bf16x2(__uint_as_float(t[8 * q + 6]), __uint_as_float(t[8 * q + 7]));
+          const int col = c0 + 8 * q;
+          *reinterpret_cast<uint4 *>(sT + (col / 64) * CHUNK_BYTES + sw128_offset(rr, (col % 64) / 8)) = v;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(ts_ready);
+    }
+    float ss = 0.f;
+    for (int nc = 0; ok && nc < nch; ++nc) {
+      const int acc = nc & 1;
+      const bool okw = mbar_wait(&acc_full[acc], (nc >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x57u);
+      if (!__all_sync(0xffffffffu, okw)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        uint32_t y[32];
+        tmem_ld32(lane_base + acc * 256 + c0, y);
+        tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          const float v = __uint_as_float(y[t]);
+          ss = fmaf(v, v, ss);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+    }
+    if (ok && m0 + rr < p.M) p.scores[m0 + rr] = sqrtf(ss);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+spts_status launch_ltp_bf16(const void *x, int64_t Nc, int D, const void *A, int r, const void *B, int Dout,
+                            float *scores, uint32_t *status, cudaStream_t s) {
+  if (Nc == 0) return SPTS_OK;
+  CUtensorMap tx, ta, tb;
+  SPTS_TRY(tmap_bf16_2d(&tx, x, static_cast<uint64_t>(Nc), D, D, 128));
+  SPTS_TRY(tmap_bf16_2d(&ta, A, r, D, D, static_cast<uint32_t>(r)));
+  SPTS_TRY(tmap_bf16_2d(&tb, B, Dout, r, r, 256));
+  Params p{static_cast<int>(Nc), D, r, Dout, scores, status, wait_limit_ns()};
+  SPTS_CUDA_TRY(
+      cudaFuncSetAttribute(ltp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM_BYTES)));
+  ltp_kernel<<<static_cast<unsigned>((Nc + 127) / 128), THREADS, SMEM_BYTES, s>>>(tx, ta, tb, p);
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+}  // namespace spts

@@ -1,0 +1,223 @@
+// rowops.cu -- HBM-bound row kernels of the layer: RMSNorm (with optional
+// row gather) to bf16, in-place rotate-half RoPE, 16-byte row gather, the
+// synthetic salient-key injection, and the per-group score reduction.
+//
+// All of these move whole rows with 16-byte vector accesses, one warp per
+// row, so a warp touches 512 contiguous bytes per instruction.
+#include "host.hpp"
+#include "rowops.cuh"
+#include "sm100.cuh"
+
+namespace spts {
+
+// ---------------------------------------------------------------- RMSNorm
+// One warp per output row; x fp32 [*, D], y bf16 [m, D].  D % 8 == 0.
+__global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const float *__restrict__ x,
+                                                           const int32_t *__restrict__ rows, int64_t m, int D,
+                                                           const __nv_bfloat16 *__restrict__ w, float eps,
+                                                           __nv_bfloat16 *__restrict__ y) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (i >= m) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t src = rows ? rows[i] : i;
+  const float4 *xr = reinterpret_cast<const float4 *>(x + src * D);
+  float ss = 0.f;
+  for (int c = lane; c < D / 4; c += 32) {
+    float4 v = __ldg(xr + c);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
+  uint4 *yr = reinterpret_cast<uint4 *>(y + i * D);
+  for (int c = lane; c < D / 8; c += 32) {
+    float4 a = __ldg(xr + 2 * c), b = __ldg(xr + 2 * c + 1);
+    float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    if (w) {
+      uint4 wv = __ldg(reinterpret_cast<const uint4 *>(w) + c);
+      const __nv_bfloat16 *wb = reinterpret_cast<const __nv_bfloat16 *>(&wv);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) v[t] = v[t] * inv * __bfloat162float(wb[t]);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) v[t] = v[t] * inv;
+    }
+    uint4 o;
+    o.x = pack_bf16x2(v[0], v[1]);
+    o.y = pack_bf16x2(v[2], v[3]);
+    o.z = pack_bf16x2(v[4], v[5]);
+    o.w = pack_bf16x2(v[6], v[7]);
+    yr[c] = o;
+  }
+}
+
+spts_status launch_rmsnorm_rows(const float *x, const int32_t *rows, int64_t m, int D, const void *w, float eps,
+                                void *y, cudaStream_t s) {
+  if (m == 0) return SPTS_OK;
+  const int64_t blocks = (m + 7) / 8;
+  rmsnorm_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      x, rows, m, D, static_cast<const __nv_bfloat16 *>(w), eps, static_cast<__nv_bfloat16 *>(y));
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+// ---------------------------------------------------------------- RoPE
+// Angle pos * inv_freq[i] is formed and reduced modulo 2*pi in fp64, then
+// sincosf runs on the reduced fp32 angle, so positions up to 2^31 keep full
+// fp32 accuracy.  One thread per (row, pair i), looping over the heads.
+__device__ __forceinline__ void rope_angle(int32_t pos, double inv_freq, float *c, float *s) {
+  const double two_pi = 6.283185307179586476925286766559;
+  double a = static_cast<double>(pos) * inv_freq;
+  a -= two_pi * rint(a / two_pi);
+  sincosf(static_cast<float>(a), s, c);
+}
+
+__global__ void rope_kernel(__nv_bfloat16 *__restrict__ x, int64_t m, int H, int d,
+                            const int32_t *__restrict__ pos, RopeFreqs f) {
+  const int half = d / 2;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= m * half) return;
+  const int64_t row = t / half;
+  const int i = static_cast<int>(t % half);
+  float c, s;
+  rope_angle(pos[row], f.inv_freq[i], &c, &s);
+  __nv_bfloat16 *xr = x + row * static_cast<int64_t>(H) * d;
+  for (int h = 0; h < H; ++h) {
+    const float x1 = __bfloat162float(xr[h * d + i]);
+    const float x2 = __bfloat162float(xr[h * d + i + half]);
+    xr[h * d + i] = __float2bfloat16_rn(x1 * c - x2 * s);
+    xr[h * d + i + half] = __float2bfloat16_rn(x2 * c + x1 * s);
+  }
+}
+
+void fill_rope_freqs(RopeFreqs *f, int d, double theta) {
+  for (int i = 0; i < d / 2 && i < 128; ++i) f->inv_freq[i] = pow(theta, -2.0 * i / d);
+}
+
+spts_status launch_rope(void *x, int64_t m, int H, int d, const int32_t *pos, double theta, cudaStream_t s) {
+  if (m == 0) return SPTS_OK;
+  RopeFreqs f;
+  fill_rope_freqs(&f, d, theta);
+  const int64_t n = m * (d / 2);
+  rope_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(static_cast<__nv_bfloat16 *>(x), m, H, d,
+                                                                      pos, f);
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+// ---------------------------------------------------------------- gather
+// One warp per destination row, 16-byte copies.  Rows outside [0, n_src)
+// are skipped and reported in the status word.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ src, int64_t n_src,
+                                                          const int32_t *__restrict__ rows, int64_t m,
+                                                          int64_t vec_per_row, uint4 *__restrict__ dst,
+                                                          const int32_t *__restrict__ pos_in,
+                                                          int32_t *__restrict__ pos_out, uint32_t *status) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (i >= m) return;
+  const int lane = threadIdx.x & 31;
+  const int32_t r = rows[i];
+  if (r < 0 || r >= n_src) {
+    if (lane == 0) raise_status(status, SPTS_DEV_BADINDEX, 0x61u, static_cast<uint32_t>(r));
+    return;
+  }
+  const uint4 *s = src + static_cast<int64_t>(r) * vec_per_row;
+  uint4 *d = dst + i * vec_per_row;
+  for (int64_t c = lane; c < vec_per_row; c += 32) d[c] = __ldg(s + c);
+  if (pos_out && lane == 0) pos_out[i] = pos_in[r];
+}
+
+spts_status launch_gather_rows(const void *src, int64_t n_src, const int32_t *rows, int64_t m, int64_t row_bytes,
+                               void *dst, const int32_t *pos_in, int32_t *pos_out, uint32_t *status,
+                               cudaStream_t s) {
+  if (m == 0) return SPTS_OK;
+  gather_rows_kernel<<<static_cast<unsigned>((m + 7) / 8), 256, 0, s>>>(
+      static_cast<const uint4 *>(src), n_src, rows, m, row_bytes / 16, static_cast<uint4 *>(dst), pos_in, pos_out,
+      status);
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+// ---------------------------------------------------------------- salience
+// Synthetic-workload step (not SPTS): K[rows[t], g] += shift * unit(mean of
+// the group's probe queries).  One block per KV head, d threads.
+__global__ void inject_salience_kernel(__nv_bfloat16 *__restrict__ k, int64_t Nc, const __nv_bfloat16 *__restrict__ q,
+                                       int P, int Hq, int Hkv, int d, const int32_t *__restrict__ rows, int64_t n_rows,
+                                       float shift, uint32_t *status) {
+  extern __shared__ float red[];
+  const int g = blockIdx.x, i = threadIdx.x, G = Hq / Hkv;
+  double acc = 0.0;
+  for (int p = 0; p < P; ++p)
+    for (int j = 0; j < G; ++j) acc += __bfloat162float(q[(static_cast<int64_t>(p) * Hq + g * G + j) * d + i]);
+  const float mean = static_cast<float>(acc / (P * G));
+  red[i] = mean * mean;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (i < o) red[i] += red[i + o];
+    __syncthreads();
+  }
+  const float u = mean / sqrtf(red[0]);
+  for (int64_t t = 0; t < n_rows; ++t) {
+    const int32_t row = rows[t];
+    if (row < 0 || row >= Nc) {
+      if (i == 0) raise_status(status, SPTS_DEV_BADINDEX, 0x62u, static_cast<uint32_t>(row));
+      continue;
+    }
+    __nv_bfloat16 *kr = k + (static_cast<int64_t>(row) * Hkv + g) * d;
+    kr[i] = __float2bfloat16_rn(__bfloat162float(kr[i]) + shift * u);
+  }
+}
+
+spts_status launch_inject_salience(void *k, int64_t Nc, const void *q_probe, int P, int Hq, int Hkv, int d,
+                                   const int32_t *rows, int64_t n_rows, float shift, uint32_t *status,
+                                   cudaStream_t s) {
+  if (n_rows == 0) return SPTS_OK;
+  inject_salience_kernel<<<Hkv, d, d * sizeof(float), s>>>(static_cast<__nv_bfloat16 *>(k), Nc,
+                                                           static_cast<const __nv_bfloat16 *>(q_probe), P, Hq,
+                                                           Hkv, d, rows, n_rows, shift, status);
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+// ---------------------------------------------------------------- group sum
+// s[j] = sum_g group[g][j], fixed order (deterministic).
+__global__ void sum_groups_kernel(const float *__restrict__ group, int G, int64_t n, float *__restrict__ s) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  float acc = 0.f;
+  for (int g = 0; g < G; ++g) acc += group[g * n + j];
+  s[j] = acc;
+}
+
+spts_status launch_sum_groups(const float *group, int G, int64_t n, float *s, cudaStream_t st) {
+  if (n == 0) return SPTS_OK;
+  sum_groups_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(group, G, n, s);
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+}  // namespace spts
+
+namespace spts {
+
+// dst[i] = src[idx[i]] for int32 vectors (positions of the selected rows).
+__global__ void gather_i32_kernel(const int32_t *__restrict__ src, const int32_t *__restrict__ idx, int64_t m,
+                                  int32_t *__restrict__ dst) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < m) dst[i] = src[idx[i]];
+}
+
+spts_status launch_gather_i32(const int32_t *src, const int32_t *idx, int64_t m, int32_t *dst, cudaStream_t s) {
+  if (m == 0) return SPTS_OK;
+  gather_i32_kernel<<<static_cast<unsigned>((m + 255) / 256), 256, 0, s>>>(src, idx, m, dst);
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+}  // namespace spts

@@ -1,0 +1,73 @@
+// rowops.cuh -- launchers of the row kernels, the top-k / prune kernels, and
+// the attention, probe, LTP and GEMM kernels (internal interface between the
+// C-ABI layer and the kernels).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "spts.h"
+
+namespace spts {
+
+struct RopeFreqs {
+  double inv_freq[128];  // theta^(-2i/d), i < d/2
+};
+void fill_rope_freqs(RopeFreqs *f, int d, double theta);
+
+spts_status launch_rmsnorm_rows(const float *x, const int32_t *rows, int64_t m, int D, const void *w, float eps,
+                                void *y, cudaStream_t s);
+spts_status launch_rope(void *x, int64_t m, int H, int d, const int32_t *pos, double theta, cudaStream_t s);
+spts_status launch_gather_rows(const void *src, int64_t n_src, const int32_t *rows, int64_t m, int64_t row_bytes,
+                               void *dst, const int32_t *pos_in, int32_t *pos_out, uint32_t *status,
+                               cudaStream_t s);
+spts_status launch_inject_salience(void *k, int64_t Nc, const void *q_probe, int P, int Hq, int Hkv, int d,
+                                   const int32_t *rows, int64_t n_rows, float shift, uint32_t *status,
+                                   cudaStream_t s);
+spts_status launch_gather_i32(const int32_t *src, const int32_t *idx, int64_t m, int32_t *dst, cudaStream_t s);
+spts_status launch_sum_groups(const float *group, int G, int64_t n, float *s, cudaStream_t st);
+
+// Top-k selection (single CTA radix select + stable compaction).
+spts_status launch_select_topk(const float *s_a, const float *s_b, int mode, float w_a, float w_b, int64_t Nc,
+                               int64_t k, int64_t force_tail, int32_t *idx_out, float *fused_out,
+                               float *kth_out, uint32_t *status, cudaStream_t s);
+
+// fp32 CUDA-core attention paths.
+spts_status launch_probe_f32(const float *q, const int32_t *qpos, int P, const float *k, const int32_t *kpos,
+                             int64_t Nc, int Hq, int Hkv, int d, float scale, float *scores, float *group,
+                             float *row_stats, cudaStream_t s);
+spts_status launch_attention_f32(const float *q, const int32_t *qpos, int64_t m, const float *k, const float *v,
+                                 const int32_t *kpos, int64_t Nc, int Hq, int Hkv, int d, float scale, float *o,
+                                 cudaStream_t s);
+
+// bf16 tensor-core paths (tcgen05).
+struct GemmArgs {
+  const void *A;
+  int64_t M;
+  int K;
+  const void *W;
+  const void *W2;
+  int N;
+  int epi;
+  void *out;
+  const int32_t *rows;
+  const int32_t *row_pos;
+  double theta;
+  uint32_t *status;
+};
+spts_status launch_gemm(const GemmArgs &g, cudaStream_t s);
+
+spts_status launch_probe_bf16(const void *q, const int32_t *qpos, int P, const void *k, const int32_t *kpos,
+                              int64_t Nc, int Hq, int Hkv, float scale, float *group, float *row_stats,
+                              uint32_t *status, cudaStream_t s);
+size_t probe_bf16_stats_bytes(int P, int Hq, int64_t Nc);
+
+spts_status launch_ltp_bf16(const void *x, int64_t Nc, int D, const void *A, int r, const void *B, int Dout,
+                            float *scores, uint32_t *status, cudaStream_t s);
+
+spts_status launch_attention_bf16(const void *q, const int32_t *qpos, int64_t m, const void *k, const void *v,
+                                  const int32_t *kpos, int64_t Nc, int Hq, int Hkv, float scale, void *o,
+                                  uint32_t *status, cudaStream_t s);
+
+}  // namespace spts
