@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of the SPTS prefill layer on B200 (tokens/s per layer, % of roofline).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+for the layer workloads a full SPTS layer (norm, K/V/Q projections, PAP probe
+scores, selection, reduced attention, O projection, LTP score, fused
+selection, reduced FFN); for ``msdp_32k`` the eight-layer MSDP pipeline with
+its four stage prunes.  Each step runs in place on the previous step's
+residual stream, so inputs stay resident in HBM; every input (h: 512 MB at
+32K, weights: 436 MB) is larger than L2, so no L2 flush is needed.
+
+Multi-GPU: the path does not shard inside one sequence, so N GPUs run N
+independent replicas (weak scaling, no data-path collective); the timed
+region is bracketed by barriers and the time is the max over ranks.
+
+``--impl reference`` times the CPU oracle (the only other implementation of
+this path) on a bounded sample of the same workload, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from synthetic import WORKLOADS, keep_rows, make_hidden, make_layer_weights, salient_rows  # noqa: E402
+
+METRIC = "prefill tokens/s per SPTS layer at 32K/128K on 1 B200; % of roofline"
+DEFAULT_STEPS = {"attn_8k": 400, "layer_32k": 200, "layer_128k": 40, "msdp_32k": 30, "layer_small": 200}
+
+
+# ---------------------------------------------------------------- peaks
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- algorithmic work
+def layer_work(wl, Nc, k, P, idx_attn, ffn=True):
+    """Algorithmic FLOPs per stage and HBM bytes of one layer.
+
+    Positions are ascending and unique, so a query at candidate index i sees
+    i + 1 keys; attention counts only those (causal) pairs.  The probe is
+    counted twice (row statistics, then column sums)."""
+    D, Hq, Hkv, d, F, r = wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r
+    vis = float(np.sum(idx_attn.astype(np.float64) + 1.0))
+    probe_vis = float(sum(Nc - P + p + 1 for p in range(P)))
+    fl = {
+        "k_proj_rope": 2.0 * Nc * D * Hkv * d,
+        "v_proj": 2.0 * Nc * D * Hkv * d,
+        "probe_q_proj": 2.0 * P * D * Hq * d,
+        "probe_scores": 2.0 * (2.0 * Hq * d * probe_vis),
+        "q_proj_rope": 2.0 * k * D * Hq * d,
+        "reduced_attention": 4.0 * Hq * d * vis,
+        "o_proj_scatter": 2.0 * k * Hq * d * D,
+    }
+    if ffn:
+        fl.update({"ltp_scores": 2.0 * Nc * (D * r + r * D), "gate_up_swiglu": 4.0 * k * D * F,
+                   "down_proj_scatter": 2.0 * k * F * D})
+    w_bytes = 2.0 * (D * Hq * d * 2 + D * Hkv * d * 2 + (3 * D * F + 2 * D * r if ffn else 0))
+    act_bytes = (Nc * D * 4 * 2 * (2 if ffn else 1)          # h read by each norm, written back
+                 + Nc * D * 2 * 2 * (2 if ffn else 1)        # normed rows written and read
+                 + Nc * Hkv * d * 2 * 2 * 2                  # K, V written and read
+                 + k * Hq * d * 2 * 4                        # Q_sel and O_sel written and read
+                 + (k * F * 2 * 2 if ffn else 0))            # SwiGLU activation written and read
+    return fl, w_bytes + act_bytes
+
+
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(value, device):
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms_max):
+    """Whole-job units per second: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1000.0)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev):
+        self.proc = None
+        self.out = tempfile.TemporaryFile(mode="w+")
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- the GPU arm
+class LayerCase:
+    """Inputs and weights of one layer workload, resident on the GPU."""
+
+    def __init__(self, S, wl, dev, layer=0):
+        self.S, self.wl = S, wl
+        self.h0 = make_hidden(wl).to(dev)
+        self.W = {n: t.to(dev) for n, t in make_layer_weights(wl, layer).items()}
+        self.pos = torch.arange(wl.N, dtype=torch.int32, device=dev)
+        self.sal = salient_rows(wl.N, wl.P, wl.salient_frac, wl.seed).to(dev)
+        self.weights = S.layer_weights(self.W)
+
+    def desc(self, k=None):
+        wl = self.wl
+        return self.S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k if k is None else k,
+                                 fuse=wl.fuse, salient_rows=self.sal if len(self.sal) else None,
+                                 salient_shift=wl.salient_shift)
+
+
+def run_msdp_step(S, wl, h, pos, layers, f_buf):
+    """The MSDP pipeline: stages of two layers, pruning at each boundary."""
+    N = wl.N
+    li = 0
+    for ratio in wl.ratios:
+        k_s = keep_rows(ratio, N)
+        Nc = h.shape[0]
+        for _ in range(2):
+            desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, k_s, fuse=wl.fuse)
+            S.spts_layer_forward(h, pos, desc, layers[li], outputs={"f": f_buf[:Nc]})
+            li += 1
+        h, pos, _ = S.spts_stage_prune(f_buf[:Nc], k_s, wl.P, h, pos)
+    return h, pos
+
+
+def gpu_arm(args, rank, world, dev):
+    import token_skipping_sparse_b200 as S
+
+    wl = WORKLOADS[args.workload]
+    peaks = measured_peaks()
+    torch.manual_seed(0)
+    msdp = bool(wl.ratios)
+    if msdp:
+        base = LayerCase(S, wl, dev, 0)
+        layer_ws = [S.layer_weights({n: t.to(dev) for n, t in make_layer_weights(wl, i).items()})
+                    for i in range(wl.layers)]
+        keep_alive = [base]
+        layer_ws_refs = layer_ws
+        f_buf = torch.empty(wl.N, dtype=torch.float32, device=dev)
+
+        def step(h):
+            return run_msdp_step(S, wl, h, base.pos, layer_ws_refs, f_buf)[0]
+    else:
+        case = LayerCase(S, wl, dev)
+        desc = case.desc()
+        keep_alive = [case]
+
+        def step(h):
+            S.spts_layer_forward(h, case.pos, desc, case.weights)
+            return h
+
+    h = (base if msdp else case).h0.clone()
+    for _ in range(args.warmup):
+        out = step(h if not msdp else (base.h0.clone()))
+    torch.cuda.synchronize()
+    S.check_device_status()
+
+    # ---------------- timed region
+    steps = args.steps
+    inputs = [base.h0.clone() for _ in range(1)] if msdp else None
+    sampler = ClockSampler(dev) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    n0 = S.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        out = step(h if not msdp else inputs[0])
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    launches = S.launch_count() - n0
+    clocks = sampler.stop() if sampler else None
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
+    S.check_device_status()
+    ms_step = ms_total / steps
+    layers_per_step = wl.layers if msdp else 1
+    value = job_throughput(wl.N * layers_per_step * steps, world, ms_total)
+
+    # ---------------- algorithmic work and per-stage breakdown (one layer)
+    lcase = base if msdp else case
+    ldesc = (S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, keep_rows(wl.ratios[0], wl.N), fuse=wl.fuse)
+             if msdp else desc)
+    hb = lcase.h0.clone()
+    idx = torch.empty(ldesc.k, dtype=torch.int32, device=dev)
+    evs = S.stage_events()
+    S.spts_layer_forward(hb, lcase.pos, ldesc, lcase.weights, outputs={"idx_attn": idx}, events=evs)
+    reps = 3
+    stage_ms = np.zeros(len(S.LAYER_STAGES))
+    for _ in range(reps):
+        S.spts_layer_forward(hb, lcase.pos, ldesc, lcase.weights, events=evs)
+        torch.cuda.synchronize()
+        stage_ms += np.array([evs[i].elapsed_time(evs[i + 1]) for i in range(len(S.LAYER_STAGES))])
+    stage_ms /= reps
+    ffn = wl.F > 0
+    fl, nbytes = layer_work(wl, wl.N, ldesc.k, wl.P, idx.cpu().numpy(), ffn)
+    kernel_stages = ["k_proj_rope", "v_proj", "q_proj_rope", "reduced_attention", "o_proj_scatter", "ltp_scores",
+                     "gate_up_swiglu", "down_proj_scatter"]
+    by_name = dict(zip(S.LAYER_STAGES, stage_ms))
+    dom = max((s for s in kernel_stages if s in fl), key=lambda s: by_name[s])
+    dom_ms = by_name[dom]
+    achieved = fl[dom] / (dom_ms / 1e3) / 1e12
+    layer_flops = sum(fl.values())
+    layer_ms = float(stage_ms.sum())
+    t_roof_ms = max(layer_flops / (peaks["bf16_sustained"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+
+    # ---------------- skipped-prefill speedup over the same kernels at keep 1.0
+    dense = None
+    if not msdp and not args.no_dense:
+        ddesc = lcase.desc(k=wl.N) if not msdp else None
+        hd = lcase.h0.clone()
+        S.spts_layer_forward(hd, lcase.pos, ddesc, lcase.weights)
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nd = 3
+        d0.record()
+        for _ in range(nd):
+            S.spts_layer_forward(hd, lcase.pos, ddesc, lcase.weights)
+        d1.record()
+        torch.cuda.synchronize()
+        dense_ms = d0.elapsed_time(d1) / nd
+        dense = {"keep": 1.0, "ms_per_layer": round(dense_ms, 4),
+                 "speedup_of_skipping": round(dense_ms / (ms_step / layers_per_step), 3)}
+        del hd
+
+    # ---------------- end to end through the C ABI with host buffers
+    e2e = None
+    if not msdp:
+        hh = torch.empty_like(lcase.h0, device="cpu").pin_memory()
+        hh.copy_(lcase.h0.cpu())
+        ho = torch.empty_like(hh).pin_memory()
+        hdv = torch.empty_like(lcase.h0)
+        ne = min(steps, 10)
+        S.spts_layer_forward(hdv.copy_(hh, non_blocking=True), lcase.pos, desc, lcase.weights)
+        ho.copy_(hdv, non_blocking=True)
+        torch.cuda.synchronize()
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record()
+        for _ in range(ne):
+            hdv.copy_(hh, non_blocking=True)
+            S.spts_layer_forward(hdv, lcase.pos, desc, lcase.weights)
+            ho.copy_(hdv, non_blocking=True)
+        x1.record()
+        torch.cuda.synchronize()
+        e2e_ms = x0.elapsed_time(x1) / ne
+        nbh = hh.numel() * hh.element_size()
+        e2e = {"value": round(wl.N * world / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": nbh,
+               "d2h_bytes_per_step": nbh, "ms_per_step": round(e2e_ms, 4)}
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) hidden states, N(0,0.02) weights)",
+        "config": {"workload": wl.name, "N": wl.N, "keep": wl.keep, "k": ldesc.k, "P": wl.P, "Hq": wl.Hq,
+                   "Hkv": wl.Hkv, "d_head": wl.d, "D": wl.D, "F": wl.F, "ltp_rank": wl.r,
+                   "layers_per_step": layers_per_step, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (no flush)", "input": "each step runs on the previous step's output"},
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_sustained"], 4), "traffic": None,
+                     "peak_note": f"{peaks['source']} sustained bf16 (kernel timed inside a long step)"},
+        "layer_roofline": {"flops": layer_flops, "hbm_bytes": nbytes, "t_roof_ms": round(t_roof_ms, 4),
+                           "ms_measured": round(ms_step / layers_per_step, 4),
+                           "frac": round(t_roof_ms / (ms_step / layers_per_step), 4),
+                           "peak_tflops": peaks["bf16_sustained"], "peak_hbm_gbs": peaks["hbm_gbs"]},
+        "stages_ms": {k: round(v, 4) for k, v in by_name.items()},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "e2e": e2e,
+        "dense_keep1": dense,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = oracle_baseline(OracleInputs(wl))
+    del keep_alive
+    return result
+
+
+# ---------------------------------------------------------------- the oracle on a bounded sample
+class OracleInputs:
+    """CPU (fp64) inputs of one layer workload plus the untimed set-up the
+    sampled oracle needs (keys for the probe over all N rows)."""
+
+    def __init__(self, wl):
+        import oracle as O
+        self.wl = wl
+        N, P = wl.N, wl.P
+        self.k = keep_rows(wl.ratios[0], N) if wl.ratios else wl.k
+        self.h = make_hidden(wl).double().numpy()
+        self.W = {n: t.float().double().numpy() for n, t in make_layer_weights(wl).items()}
+        self.pos = np.arange(N)
+        self.sal = salient_rows(N, P, wl.salient_frac, wl.seed).numpy()
+        xn = O.bf16_round(O.rmsnorm(self.h, None, 1e-5))
+        self.kk = O.bf16_round(O.rope((xn @ self.W["w_k"].T).reshape(N, wl.Hkv, wl.d), self.pos))
+        self.vv = O.bf16_round((xn @ self.W["w_v"].T).reshape(N, wl.Hkv, wl.d))
+        self.xn_tail = xn[N - P:]
+        self.c = O.ltp_scores(xn, self.W["ltp_a"], self.W["ltp_b"]) if wl.F else None
+
+
+def oracle_baseline(inp, row_sample=1024, sel_sample=16):
+    """Times the CPU oracle on a bounded sample of one layer.
+
+    Steps that are linear in the rows (RMSNorm, K/V projections with RoPE,
+    the LTP proxy) run on `row_sample` rows and are scaled to N; the PAP
+    probe scores and both selections run on all N rows; the per-selected-row
+    steps (Q projection, reduced attention, O projection, reduced FFN) run on
+    `sel_sample` of the k selected rows and are scaled to k."""
+    import oracle as O
+
+    wl, W, h, pos = inp.wl, inp.W, inp.h, inp.pos
+    N, P, k, Hq, Hkv, d = wl.N, wl.P, inp.k, wl.Hq, wl.Hkv, wl.d
+    rs = min(row_sample, N)
+    t0 = time.perf_counter()
+    xs = O.bf16_round(O.rmsnorm(h[:rs], None, 1e-5))
+    O.bf16_round(O.rope((xs @ W["w_k"].T).reshape(rs, Hkv, d), pos[:rs]))
+    O.bf16_round((xs @ W["w_v"].T).reshape(rs, Hkv, d))
+    if wl.F:
+        O.ltp_scores(O.bf16_round(O.rmsnorm(h[:rs], None, 1e-5)), W["ltp_a"], W["ltp_b"])
+    t_lin = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    qp = O.bf16_round(O.rope((inp.xn_tail @ W["w_q"].T).reshape(P, Hq, d), pos[N - P:]))
+    kk = O.inject_salience(inp.kk, qp, inp.sal, wl.salient_shift, Hkv) if len(inp.sal) else inp.kk
+    s, _ = O.probe_scores(qp, pos[N - P:], kk, pos)
+    idx, _ = O.select_topk(s.astype(np.float32), k, P)
+    if wl.F:
+        f = O.fuse_scores(s.astype(np.float32), inp.c.astype(np.float32), wl.fuse)
+        O.select_topk(f, k, P)
+    t_all = time.perf_counter() - t1
+    rows = idx[np.linspace(0, len(idx) - 1, sel_sample).astype(int)]
+    t2 = time.perf_counter()
+    xr = O.bf16_round(O.rmsnorm(h[rows], None, 1e-5))
+    qs = O.bf16_round(O.rope((xr @ W["w_q"].T).reshape(len(rows), Hq, d), pos[rows]))
+    o = O.bf16_round(O.reduced_attention(qs, pos[rows], kk, inp.vv, pos))
+    h1 = h[rows] + o.reshape(len(rows), -1) @ W["w_o"].T
+    if wl.F:
+        O.reduced_ffn(h1, np.arange(len(rows)), None, 1e-5, W["w_gate"], W["w_up"], W["w_down"])
+    t_sel = time.perf_counter() - t2
+    total = t_lin * (N / rs) + t_all + t_sel * (k / len(rows))
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return {"value": round(N / total, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"{wl.name}: row-linear steps on {rs} of {N} rows ({t_lin:.2f} s, scaled x{N / rs:.0f}); "
+                       f"probe scores and selections on all {N} rows ({t_all:.2f} s); per-selected-row steps "
+                       f"on {len(rows)} of {k} rows ({t_sel:.2f} s, scaled x{k / len(rows):.0f}); fp64 numpy"),
+            "seconds": round(t_lin + t_all + t_sel, 2), "est_seconds_per_layer": round(total, 2)}
+
+
+def reference_arm(args):
+    wl = WORKLOADS[args.workload]
+    inp = OracleInputs(wl)
+    for _ in range(args.warmup):
+        oracle_baseline(inp)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(oracle_baseline(inp))
+    wall = time.perf_counter() - t0
+    v = statistics.median([x["value"] for x in vals])
+    cb = dict(vals[-1])
+    cb["value"] = v
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * wall / max(1, args.steps), 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "N": wl.N, "keep": wl.keep, "P": wl.P},
+            "cpu_baseline": cb, "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="layer_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS.get(args.workload, 50) if args.impl == "ours" else 3
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args)), flush=True)
+        return 0
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=dev)
+    try:
+        res = gpu_arm(args, rank, world, dev)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

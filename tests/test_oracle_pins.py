@@ -330,6 +330,22 @@ def test_msdp_all_ratios_one_is_dense_stack_and_sets_nest():
     assert set(opos.tolist()) == seen and {pos[-1], pos[-2]} <= seen
 
 
+# ---------------------------------------------------------------- synthetic salience
+def test_inject_salience_closed_form():
+    # two probes x two heads of one KV group: mean (0.5, 0.5, 0, 0) -> unit (1, 1, 0, 0)/sqrt(2)
+    q = np.zeros((2, 2, 4))
+    q[0, :, 0] = 1.0
+    q[1, :, 1] = 1.0
+    k = np.zeros((5, 1, 4))
+    k[:, 0, 3] = 0.5
+    out = O.inject_salience(k, q, np.array([1, 3]), 3.0, 1)
+    add = 3.0 / math.sqrt(2.0)
+    want = k.copy()
+    want[[1, 3], 0, 0] = torch.tensor(add, dtype=torch.float32).to(torch.bfloat16).item()
+    want[[1, 3], 0, 1] = want[1, 0, 0]
+    np.testing.assert_array_equal(out, want)
+
+
 # ---------------------------------------------------------------- accounting
 def _golden(golden_dir, name):
     rows = []

@@ -339,10 +339,14 @@ def spts_layer_forward(h, pos, desc, weights, outputs=False, ws=None, events=Non
     ev_arr = None
     if events is not None:
         ev_arr = (C.c_void_p * LAYER_STAGE_EVENTS)(*[e.cuda_event for e in events])
-    if outputs or events is not None:
+    if outputs is not False or events is not None:
         out = LayerOutputs()
         out.stage_events = C.cast(ev_arr, C.c_void_p) if ev_arr is not None else None
-    if outputs:
+    if isinstance(outputs, dict):          # caller-provided subset of the outputs
+        res = outputs
+        for n, t in res.items():
+            setattr(out, n, t.data_ptr())
+    elif outputs:
         dv = h.device
         k, hq = desc.k, desc.Hq * desc.d
         res = dict(s=torch.empty(Nc, dtype=torch.float32, device=dv),
