@@ -196,6 +196,29 @@ SPTS_API spts_status spts_stage_prune(const float *scores, int64_t Nc, int64_t k
                              spts_stream stream);
 SPTS_API size_t spts_stage_prune_workspace(int64_t Nc);
 
+/* Allocation-free variant of spts_stage_prune.  The paper has no
+ * counterpart; this exists for callers that cannot allocate device memory
+ * when they call in (a plugin inside a host framework that reserved the GPU's
+ * memory up front and forbids further cudaMalloc, or a latency-critical loop
+ * that cannot take cudaMalloc's implicit synchronisation).  Same arguments
+ * and results as spts_stage_prune, without the workspace: when kept_idx is
+ * NULL the kept indices go to a fixed device array inside the library
+ * (SPTS_NOALLOC_MAX_NC int32, 1 MiB, held by every GPU that loads the library
+ * until the process exits).
+ *  - Nc > SPTS_NOALLOC_MAX_NC returns SPTS_ERR_SHAPE.
+ *  - Calls nothing that allocates (no cudaMalloc/cudaFree).  The first call
+ *    on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array, which keeps the last call's contents:
+ *    calls that may overlap on the GPU (different streams, or different host
+ *    threads on one device) race on it and must be serialised by the caller.
+ *  - Device-side checks (non-finite scores) are not reported by this variant. */
+#define SPTS_NOALLOC_MAX_NC 262144
+SPTS_API spts_status spts_stage_prune_noalloc(const float *scores, int64_t Nc, int64_t k_keep, int64_t force_tail,
+                                              const float *h_in, const int32_t *pos_in, int D, float *h_out,
+                                              int32_t *pos_out, int32_t *kept_idx, spts_stream stream);
+
 /* ---------------------------------------------------------------------- */
 /* Supporting calls used to compose the layer                             */
 /* ---------------------------------------------------------------------- */

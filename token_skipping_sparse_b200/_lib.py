@@ -29,7 +29,7 @@ EXPORTS = (
     "spts_probe_scores", "spts_probe_scores_workspace", "spts_ltp_scores", "spts_ltp_scores_workspace",
     "spts_select_topk", "spts_select_topk_workspace", "spts_reduced_attention",
     "spts_reduced_attention_workspace", "spts_reduced_ffn", "spts_reduced_ffn_workspace", "spts_stage_prune",
-    "spts_stage_prune_workspace", "spts_rmsnorm_rows", "spts_rope", "spts_gather_rows", "spts_linear",
+    "spts_stage_prune_workspace", "spts_stage_prune_noalloc", "spts_rmsnorm_rows", "spts_rope", "spts_gather_rows", "spts_linear",
     "spts_linear_workspace", "spts_inject_salience", "spts_layer_forward", "spts_layer_forward_workspace",
 )
 
@@ -105,6 +105,8 @@ _sig("spts_reduced_ffn", i32, [i32, vp, i64, i32, vp, i64, vp, f32, vp, vp, vp, 
 _sig("spts_reduced_ffn_workspace", sz, [i64, i32, i32])
 _sig("spts_stage_prune", i32, [vp, i64, i64, i64, vp, vp, i32, vp, vp, vp, vp, sz, vp])
 _sig("spts_stage_prune_workspace", sz, [i64])
+_sig("spts_stage_prune_noalloc", i32, [vp, i64, i64, i64, vp, vp, i32, vp, vp, vp, vp])
+NOALLOC_MAX_NC = 262144
 _sig("spts_rmsnorm_rows", i32, [vp, vp, i64, i32, vp, f32, vp, vp])
 _sig("spts_rope", i32, [vp, i64, i32, i32, vp, f64, vp])
 _sig("spts_gather_rows", i32, [vp, i64, vp, i64, i64, vp, vp, vp])
@@ -258,6 +260,19 @@ def spts_stage_prune(scores, k_keep, force_tail, h, pos, ws=None):
     check(lib.spts_stage_prune(ptr(scores), Nc, k_keep, force_tail, ptr(h), ptr(pos), D, ptr(h_out),
                                ptr(pos_out), ptr(kept), ptr(ws), ws.numel(), stream_ptr()))
     return h_out, pos_out, kept
+
+
+def spts_stage_prune_noalloc(scores, k_keep, force_tail, h, pos, kept=None):
+    """The allocation-free stage prune: no workspace; the kept indices go to
+    the library's fixed device array unless `kept` (int32 [k_keep]) is given.
+    Output tensors are allocated here by torch, as for every call of this
+    binding; the C entry point itself allocates nothing."""
+    Nc, D = h.shape
+    h_out = torch.empty(k_keep, D, dtype=h.dtype, device=h.device)
+    pos_out = torch.empty(k_keep, dtype=torch.int32, device=h.device)
+    check(lib.spts_stage_prune_noalloc(ptr(scores), Nc, k_keep, force_tail, ptr(h), ptr(pos), D, ptr(h_out),
+                                       ptr(pos_out), ptr(kept), stream_ptr()))
+    return h_out, pos_out
 
 
 # ---------------------------------------------------------------- supporting calls
