@@ -322,6 +322,28 @@ SPTS_API spts_status spts_layer_forward(const spts_layer_desc *L, const spts_lay
                                size_t ws_bytes, spts_stream stream);
 SPTS_API size_t spts_layer_forward_workspace(const spts_layer_desc *L, int64_t Nc);
 
+/* Multi-Stage Delayed Pruning over a stack of layers (SPTS, Fig. 2(c),
+ * Fig. A, Table B).  n_stages stages of layers_per_stage layers each
+ * (n_layers = n_stages * layers_per_stage).  Stage s starts with candidate
+ * set C_s (C_1 = all N rows); every layer of the stage runs spts_layer_forward
+ * on C_s with k = stage_k[s] active rows; at the end of the stage C_{s+1} =
+ * the top stage_k[s] rows of C_s by the fused FFN-selection score of the
+ * stage's last layer (last P rows kept), compacted in ascending order.
+ *   L           layer geometry (L->k is ignored; stage_k gives each stage's k)
+ *   W           [n_layers] weights, one entry per layer
+ *   stage_k     [n_stages] host array, P <= stage_k[s] <= size of C_s
+ *   h           [N, D] fp32 in/out: on return rows [0, stage_k[last]) hold
+ *               the final candidates' hidden states (other rows: scratch)
+ *   pos         [N] int32 in/out, likewise compacted
+ *   stage_pos   nullable, [sum_s stage_k[s]] int32 out: positions of C_{s+1}
+ *               for every stage, concatenated
+ * Synthetic salience (L->n_salient) is not applied in this call. */
+SPTS_API spts_status spts_msdp_forward(const spts_layer_desc *L, const spts_layer_weights *W, int n_layers,
+                                       int layers_per_stage, const int64_t *stage_k, int n_stages, float *h,
+                                       int32_t *pos, int64_t N, int32_t *stage_pos, void *ws, size_t ws_bytes,
+                                       spts_stream stream);
+SPTS_API size_t spts_msdp_forward_workspace(const spts_layer_desc *L, int64_t N);
+
 #ifdef __cplusplus
 }
 #endif

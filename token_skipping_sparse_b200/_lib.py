@@ -31,6 +31,7 @@ EXPORTS = (
     "spts_reduced_attention_workspace", "spts_reduced_ffn", "spts_reduced_ffn_workspace", "spts_stage_prune",
     "spts_stage_prune_workspace", "spts_stage_prune_noalloc", "spts_rmsnorm_rows", "spts_rope", "spts_gather_rows", "spts_linear",
     "spts_linear_workspace", "spts_inject_salience", "spts_layer_forward", "spts_layer_forward_workspace",
+    "spts_msdp_forward", "spts_msdp_forward_workspace",
 )
 
 
@@ -117,6 +118,9 @@ if hasattr(lib, "spts_layer_forward"):
     _sig("spts_layer_forward", i32, [C.POINTER(LayerDesc), C.POINTER(LayerWeights), vp, vp, i64,
                                      C.POINTER(LayerOutputs), vp, sz, vp])
     _sig("spts_layer_forward_workspace", sz, [C.POINTER(LayerDesc), i64])
+    _sig("spts_msdp_forward", i32, [C.POINTER(LayerDesc), C.POINTER(LayerWeights), i32, i32, C.POINTER(C.c_int64),
+                                    i32, vp, vp, i64, vp, vp, sz, vp])
+    _sig("spts_msdp_forward_workspace", sz, [C.POINTER(LayerDesc), i64])
 
 
 # ---------------------------------------------------------------- helpers
@@ -379,3 +383,25 @@ def spts_layer_forward(h, pos, desc, weights, outputs=False, ws=None, events=Non
     check(lib.spts_layer_forward(C.byref(desc), C.byref(w), ptr(h), ptr(pos), Nc,
                                  None if out is None else C.byref(out), ptr(ws), ws.numel(), stream_ptr()))
     return res
+
+
+def spts_msdp_forward(h, pos, desc, layer_weights_list, layers_per_stage, stage_k, stage_pos=False, ws=None):
+    """MSDP over len(layer_weights_list) layers, in place on h [N, D] / pos [N].
+    Returns (number of final candidates, per-stage candidate positions or None)."""
+    N = h.shape[0]
+    n_layers = len(layer_weights_list)
+    ws_list = [w if isinstance(w, LayerWeights) else layer_weights(w) for w in layer_weights_list]
+    W = (LayerWeights * n_layers)(*ws_list)
+    ks = (C.c_int64 * len(stage_k))(*[int(k) for k in stage_k])
+    sp = torch.empty(int(sum(stage_k)), dtype=torch.int32, device=h.device) if stage_pos else None
+    n = lib.spts_msdp_forward_workspace(C.byref(desc), N)
+    ws = workspace(n) if ws is None else ws
+    check(lib.spts_msdp_forward(C.byref(desc), W, n_layers, layers_per_stage, ks, len(stage_k), ptr(h), ptr(pos),
+                                N, ptr(sp), ptr(ws), ws.numel(), stream_ptr()))
+    if sp is None:
+        return int(stage_k[-1]), None
+    out, off = [], 0
+    for k in stage_k:
+        out.append(sp[off:off + int(k)])
+        off += int(k)
+    return int(stage_k[-1]), out

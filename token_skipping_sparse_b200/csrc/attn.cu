@@ -6,15 +6,19 @@
 // G query heads that share KV head g (G = Hq/Hkv), so every K/V tile loaded
 // serves all G heads in one M=128 MMA.
 //   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys into a
-//               2-stage ring (128-byte swizzle);
+//               3-stage ring (128-byte swizzle);
 //   warp 1      MMA: S = Q K^T into one of two TMEM buffers (M=128, N=128,
-//               K=128), then O += P V (P K-major from shared memory, V
-//               MN-major) into a third TMEM region;
+//               K=128), then O += P V with P read from TMEM (the softmax
+//               writes it over the S values it consumed) and V an MN-major
+//               shared-memory operand, into a third TMEM region;
 //   warps 2..5  softmax, one thread per Q row: tcgen05.ld of its S row,
-//               causal mask (only on tiles that cross the diagonal), online
-//               max with lazy rescaling (O in TMEM is rescaled only when the
-//               running max grows by more than 2^8), exp2, bf16 P written in
-//               the UMMA K-major swizzled layout; at the end O / l -> bf16.
+//               causal mask (only on tiles that cross the diagonal), row max
+//               with independent accumulators, lazy rescaling of O in TMEM
+//               (only when the running max grows by more than 2^8), exp2 with
+//               the scale folded into one FFMA, bf16 P stored back to TMEM
+//               with tcgen05.st; at the end O / l -> bf16.
+// Keeping P in TMEM takes it off the shared-memory path: per key tile the
+// shared memory then serves only the K and V tiles (TMA in, MMA out).
 // The key loop stops at the last key visible to the tile's latest query, and
 // tiles are launched latest-first so the long ones start early.
 // All barrier waits are bounded (see sm100.cuh).
@@ -29,15 +33,15 @@ namespace {
 
 constexpr int THREADS = 192;
 constexpr int BKV = 128;
+constexpr int KV_STAGES = 3;
 constexpr int TILE_BYTES = 128 * 128 * 2;  // 32 KB: 128 rows x 128 bf16, as two 64-wide swizzled chunks
 constexpr int CHUNK_BYTES = 128 * 64 * 2;  // 16 KB
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + TILE_BYTES;       // 2 stages
-constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;   // 2 stages
-constexpr int OFF_P = OFF_V + 2 * TILE_BYTES;   // 2 buffers
-constexpr int OFF_BAR = OFF_P + 2 * TILE_BYTES;
-constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 256;
-constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256,384)
+constexpr int OFF_K = OFF_Q + TILE_BYTES;               // KV_STAGES stages
+constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;   // KV_STAGES stages
+constexpr int OFF_BAR = OFF_V + KV_STAGES * TILE_BYTES;
+constexpr size_t SMEM_BYTES = OFF_BAR + 256;
+constexpr uint32_t TMEM_COLS = 512;  // S/P buffers [0,128) and [128,256), O [256,384)
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
 struct Params {
@@ -69,16 +73,14 @@ __device__ __forceinline__ int upper_bound(const int32_t *a, int n, int32_t v) {
 __global__ void __launch_bounds__(THREADS, 1)
     attention_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t *sQ = smem + OFF_Q;
   uint8_t *sK = smem + OFF_K;
   uint8_t *sV = smem + OFF_V;
-  uint8_t *sP = smem + OFF_P;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-  uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = bars + 3, *kv_empty = bars + 5, *s_full = bars + 7,
-           *p_ready = bars + 9, *p_free = bars + 11, *drain = bars + 13;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 14);
+  uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = k_full + KV_STAGES, *kv_empty = v_full + KV_STAGES,
+           *s_full = kv_empty + KV_STAGES, *p_ready = s_full + 2, *p_free = p_ready + 2, *drain = p_free + 2;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
   int *s_range = reinterpret_cast<int *>(tmem_holder + 2);  // kv_end, mask_from
 
@@ -87,12 +89,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int g = static_cast<int>(blockIdx.x) % p.Hkv;
   const int t0 = qt * p.tq;
 
+  // The swizzled operand layouts need a 1024-byte aligned base.
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) raise_status(p.status, SPTS_DEV_BADINDEX, 0x2Fu, smem_u32(smem));
+    return;
+  }
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KV_STAGES; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
       mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&p_ready[s], 128);
       mbar_init(&p_free[s], 1);
@@ -126,8 +135,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_load_3d(sQ + CHUNK_BYTES, &tmQ, q_full, 64, g * p.G, t0);
       uint32_t issued = 0, issued_par = 0;
       for (int j = 0; j < n_tiles; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
+        const int st = j % KV_STAGES;
+        const uint32_t ph = (j / KV_STAGES) & 1;
         if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_flag, p.status, p.wait_ns, 0x21u)) break;
         mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
         tma_load_3d(sK + st * TILE_BYTES, &tmK, &k_full[st], 0, g, j * BKV);
@@ -140,7 +149,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (*abort_flag) {
         mbar_drain(q_full, 0, p.status);
-        for (int st = 0; st < 2; ++st)
+        for (int st = 0; st < KV_STAGES; ++st)
           if (issued & (1u << st)) {
             mbar_drain(&k_full[st], (issued_par >> st) & 1u, p.status);
             mbar_drain(&v_full[st], (issued_par >> st) & 1u, p.status);
@@ -155,36 +164,37 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status, p.wait_ns, 0x22u);
       tc_fence_after();
       const uint32_t q_addr = smem_u32(sQ);
+      // S_j goes to TMEM buffer j % 2.  tcgen05.mma from this thread run in
+      // issue order, so S_{j+2} (issued after PV_j) cannot overwrite P_j
+      // before PV_j has read it.
       auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&k_full[st], (j >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x23u)) return false;
+        const int st = j % KV_STAGES;
+        if (!mbar_wait(&k_full[st], (j / KV_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x23u)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(sK + st * TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t a = sdesc_k_sw128(q_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3);
           const uint64_t b = sdesc_k_sw128(k_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3);
-          mma_bf16_ss(tmem + st * BKV, a, b, idesc_s, kk > 0);
+          mma_bf16_ss(tmem + (j & 1) * BKV, a, b, idesc_s, kk > 0);
         }
-        tc_commit(&s_full[st]);
+        tc_commit(&s_full[j & 1]);
         return true;
       };
       if (ok && n_tiles > 0) ok = issue_s(0);
       for (int j = 0; ok && j < n_tiles; ++j) {
         if (j + 1 < n_tiles && !issue_s(j + 1)) break;
-        const int b = j & 1;
+        const int b = j & 1, st = j % KV_STAGES;
         if (!mbar_wait(&p_ready[b], (j >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x24u)) break;
-        if (!mbar_wait(&v_full[b], (j >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x25u)) break;
+        if (!mbar_wait(&v_full[st], (j / KV_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x25u)) break;
         tc_fence_after();
-        const uint32_t p_addr = smem_u32(sP + b * TILE_BYTES);
-        const uint32_t v_addr = smem_u32(sV + b * TILE_BYTES);
+        const uint32_t v_addr = smem_u32(sV + st * TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sdesc_k_sw128(p_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3);
           const uint64_t v = sdesc_mn_sw128(v_addr + kk * 16 * 128, CHUNK_BYTES);
-          mma_bf16_ss(tmem + 256, a, v, idesc_pv, (j | kk) != 0);
+          mma_bf16_ts(tmem + 256, tmem + b * BKV + kk * 8, v, idesc_pv, (j | kk) != 0);
         }
-        tc_commit(&kv_empty[b]);
+        tc_commit(&kv_empty[st]);
         tc_commit(&p_free[b]);
       }
       tc_commit(drain);
@@ -199,6 +209,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool valid = tok < p.m;
     const int32_t qp = valid ? p.qpos[tok] : INT_MIN;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float c2 = p.scale_log2;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
@@ -214,27 +225,26 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int c = 0; c < 4; ++c)
         tmem_ld32(lane_base + b * BKV + c * 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32 * c));
       tmem_ld_wait();
+      // raw scores; the scale (> 0) is folded into the row max and the exp2 FFMA
       float x[BKV];
 #pragma unroll
       for (int c = 0; c < BKV; ++c) x[c] = __uint_as_float(xr[c]);
       const int j0 = j * BKV;
       const bool need_mask = (j0 + BKV > mask_from) || (j0 + BKV > kv_end);
-      float mt = -INFINITY;
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < BKV; ++c) {
           const int key = j0 + c;
-          const bool vis = key < kv_end && __ldg(p.kpos + key) <= qp;
-          x[c] = vis ? x[c] * p.scale_log2 : -INFINITY;
-          mt = fmaxf(mt, x[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < BKV; ++c) {
-          x[c] *= p.scale_log2;
-          mt = fmaxf(mt, x[c]);
+          if (!(key < kv_end && __ldg(p.kpos + key) <= qp)) x[c] = -INFINITY;
         }
       }
+      float m8[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) m8[t] = x[t];
+#pragma unroll
+      for (int c = 8; c < BKV; ++c) m8[c & 7] = fmaxf(m8[c & 7], x[c]);
+      const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * c2;
       const float m_new = fmaxf(m_run, mt);
       const bool need = m_new > m_run + RESCALE_THRESHOLD;
       if (__any_sync(0xffffffffu, need)) {
@@ -261,37 +271,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         l *= factor;
         m_run = m_new;
       }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // the P buffer b was last read by PV_{j-2}
-      if (j >= 2) {
-        const bool okw = mbar_wait(&p_free[b], ((j - 2) >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x28u);
-        if (!__all_sync(0xffffffffu, okw)) {
-          ok = false;
-          break;
+      const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          const float e0 = ex2(fmaf(x[h * 64 + 2 * t], c2, neg_m));
+          const float e1 = ex2(fmaf(x[h * 64 + 2 * t + 1], c2, neg_m));
+          s8[(2 * t) & 7] += e0;
+          s8[(2 * t + 1) & 7] += e1;
+          pk[t] = pack_bf16x2(e0, e1);
         }
+        // P over the S values of this buffer: columns [b*128 + 32h, +32) hold keys [64h, 64h+64)
+        tmem_st32(lane_base + b * BKV + h * 32, pk);
       }
-      uint8_t *prow = sP + b * TILE_BYTES;
-      float lsum = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          float e[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            e[t] = ex2(x[ch * 64 + u * 8 + t] - m_use);
-            lsum += e[t];
-          }
-          uint4 v;
-          v.x = pack_bf16x2(e[0], e[1]);
-          v.y = pack_bf16x2(e[2], e[3]);
-          v.z = pack_bf16x2(e[4], e[5]);
-          v.w = pack_bf16x2(e[6], e[7]);
-          *reinterpret_cast<uint4 *>(prow + ch * CHUNK_BYTES + sw128_offset(r, u)) = v;
-        }
-      }
-      l += lsum;
-      fence_proxy_async_smem();
+      l += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[b]);
     }

@@ -68,11 +68,14 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float *v
   }
 }
 
+// Angle pos * inv_freq reduced to [-pi, pi] in fp64; the fast sine/cosine of
+// the reduced fp32 angle is accurate to ~1e-6, far below bf16 resolution.
 __device__ __forceinline__ void rope_angle_f(int32_t pos, double inv_freq, float *c, float *s) {
   const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
   double a = static_cast<double>(pos) * inv_freq;
-  a -= two_pi * rint(a / two_pi);
-  sincosf(static_cast<float>(a), s, c);
+  a = fma(-two_pi, rint(a * inv_two_pi), a);
+  __sincosf(static_cast<float>(a), s, c);
 }
 
 template <int EPI>

@@ -2,6 +2,7 @@
 // of Fig. 2: probe (PAP) -> select -> reduced attention -> O projection into
 // the selected rows -> LTP score -> fuse + select -> reduced FFN.
 #include <cstring>
+#include <utility>
 
 #include "host.hpp"
 #include "rowops.cuh"
@@ -162,6 +163,75 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   GemmArgs g2{b.act, k, L->F, W->w_down, nullptr, D, SPTS_EPI_SCATTER_ADD, h, idx_f, nullptr, 0.0, st};
   SPTS_TRY(launch_gemm(g2, s));
   return mark(15);
+}
+
+// ---------------------------------------------------------------- MSDP
+size_t spts_msdp_forward_workspace(const spts_layer_desc *L, int64_t N) {
+  if (L == nullptr || N <= 0) return kStatusBytes;
+  spts_layer_desc l = *L;
+  l.k = N;  // the largest k any stage can use
+  const size_t lw = Carver::round(spts_layer_forward_workspace(&l, N));
+  return lw + Carver::round(static_cast<size_t>(N) * L->D * 4) + 3 * Carver::round(static_cast<size_t>(N) * 4);
+}
+
+spts_status spts_msdp_forward(const spts_layer_desc *L, const spts_layer_weights *W, int n_layers,
+                              int layers_per_stage, const int64_t *stage_k, int n_stages, float *h, int32_t *pos,
+                              int64_t N, int32_t *stage_pos, void *ws, size_t ws_bytes, spts_stream stream) {
+  const char *who = "spts_msdp_forward";
+  SPTS_REQUIRE(L && W && stage_k && h && pos, SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(n_stages >= 1 && layers_per_stage >= 1 && n_layers == n_stages * layers_per_stage, SPTS_ERR_SHAPE,
+               "%s: need n_layers == n_stages * layers_per_stage", who);
+  int64_t prev = N;
+  for (int s = 0; s < n_stages; ++s) {
+    SPTS_REQUIRE(stage_k[s] >= L->P && stage_k[s] <= prev, SPTS_ERR_SHAPE,
+                 "%s: stage %d keeps %lld rows of %lld (need P <= k_s <= |C_s|)", who, s,
+                 static_cast<long long>(stage_k[s]), static_cast<long long>(prev));
+    prev = stage_k[s];
+  }
+  SPTS_REQUIRE(L->F > 0, SPTS_ERR_SHAPE, "%s: pruning uses the fused FFN score, so F must be > 0", who);
+  SPTS_TRY(check_ws(ws, ws_bytes, spts_msdp_forward_workspace(L, N), who));
+  spts_layer_desc lmax = *L;
+  lmax.k = N;
+  const size_t lw = Carver::round(spts_layer_forward_workspace(&lmax, N));
+  char *extra = static_cast<char *>(ws) + lw;
+  float *h2 = reinterpret_cast<float *>(extra);
+  extra += Carver::round(static_cast<size_t>(N) * L->D * 4);
+  int32_t *pos2 = reinterpret_cast<int32_t *>(extra);
+  extra += Carver::round(static_cast<size_t>(N) * 4);
+  float *f = reinterpret_cast<float *>(extra);
+  extra += Carver::round(static_cast<size_t>(N) * 4);
+  int32_t *kept = reinterpret_cast<int32_t *>(extra);
+  uint32_t *st = static_cast<uint32_t *>(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  float *ha = h, *hb = h2;
+  int32_t *pa = pos, *pb = pos2;
+  int64_t Nc = N, out_off = 0;
+  int li = 0;
+  for (int stg = 0; stg < n_stages; ++stg) {
+    spts_layer_desc d = *L;
+    d.k = stage_k[stg];
+    d.n_salient = 0;
+    d.salient_rows = nullptr;
+    spts_layer_outputs o;
+    memset(&o, 0, sizeof(o));
+    o.f = f;
+    for (int l = 0; l < layers_per_stage; ++l, ++li) SPTS_TRY(spts_layer_forward(&d, &W[li], ha, pa, Nc, &o, ws, lw, stream));
+    // stage boundary: C_{s+1} = top-k_s of C_s by the last layer's fused score
+    SPTS_TRY(launch_select_topk(f, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, Nc, d.k, L->P, kept, nullptr, nullptr, st, s));
+    SPTS_TRY(launch_gather_rows(ha, Nc, kept, d.k, static_cast<int64_t>(L->D) * 4, hb, pa, pb, st, s));
+    if (stage_pos)
+      SPTS_CUDA_TRY(cudaMemcpyAsync(stage_pos + out_off, pb, static_cast<size_t>(d.k) * 4, cudaMemcpyDeviceToDevice, s));
+    out_off += d.k;
+    std::swap(ha, hb);
+    std::swap(pa, pb);
+    Nc = d.k;
+  }
+  if (ha != h) {
+    SPTS_CUDA_TRY(cudaMemcpyAsync(h, ha, static_cast<size_t>(Nc) * L->D * 4, cudaMemcpyDeviceToDevice, s));
+    SPTS_CUDA_TRY(cudaMemcpyAsync(pos, pa, static_cast<size_t>(Nc) * 4, cudaMemcpyDeviceToDevice, s));
+  }
+  return SPTS_OK;
 }
 
 }  // extern "C"

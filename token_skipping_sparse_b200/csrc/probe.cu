@@ -189,7 +189,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(&s_free[b]);
       const int j0 = (kt0 + i) * BKEY;
       const bool need_mask = (j0 + BKEY > mask_from) || (j0 + BKEY > kv_end);
-      float x[BKEY], mt = -INFINITY;
+      float x[BKEY], m8[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) m8[t] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < BKEY; ++c) {
         float v = __uint_as_float(xr[c]) * p.scale_log2;
@@ -198,13 +200,16 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!(key < kv_end && __ldg(p.kpos + key) <= qp)) v = -INFINITY;
         }
         x[c] = v;
-        mt = fmaxf(mt, v);
+        m8[c & 7] = fmaxf(m8[c & 7], v);
       }
+      const float mt =
+          fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float m_new = fmaxf(m, mt);
       if (m_new == -INFINITY) continue;
-      float sum = 0.f;
+      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < BKEY; ++c) sum += ex2(x[c] - m_new);
+      for (int c = 0; c < BKEY; ++c) s8[c & 7] += ex2(x[c] - m_new);
+      const float sum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
       l = (m == -INFINITY ? 0.f : l * ex2(m - m_new)) + sum;
       m = m_new;
     }
@@ -376,7 +381,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool live = j < kv_end;
       const int32_t kp = live ? __ldg(p.kpos + j) : INT_MAX;
       const bool all_vis = kp <= ppos_min;
-      float acc = 0.f;
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
       for (int c0 = 0; c0 < ncol; c0 += 32) {
         uint32_t xr[32];
@@ -385,11 +390,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
           const float2 st = sstat[c0 + t];
-          float w = ex2(__uint_as_float(xr[t]) * p.scale_log2 - st.x) * st.y;
+          float w = ex2(fmaf(__uint_as_float(xr[t]), p.scale_log2, -st.x)) * st.y;
           if (!all_vis && kp > scol[c0 + t]) w = 0.f;
-          acc += w;
+          a4[t & 3] += w;
         }
       }
+      const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
       tc_fence_before();
       mbar_arrive(&s_free[b]);
       if (live) group[static_cast<int64_t>(g) * p.Nc + j] = acc;

@@ -63,14 +63,15 @@ spts_status launch_rmsnorm_rows(const float *x, const int32_t *rows, int64_t m, 
 }
 
 // ---------------------------------------------------------------- RoPE
-// Angle pos * inv_freq[i] is formed and reduced modulo 2*pi in fp64, then
-// sincosf runs on the reduced fp32 angle, so positions up to 2^31 keep full
-// fp32 accuracy.  One thread per (row, pair i), looping over the heads.
+// Angle pos * inv_freq[i] is formed and reduced modulo 2*pi in fp64, then the
+// fast sine/cosine runs on the reduced fp32 angle (error ~1e-6 for positions
+// up to 2^31).  One thread per (row, pair i), looping over the heads.
 __device__ __forceinline__ void rope_angle(int32_t pos, double inv_freq, float *c, float *s) {
   const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
   double a = static_cast<double>(pos) * inv_freq;
-  a -= two_pi * rint(a / two_pi);
-  sincosf(static_cast<float>(a), s, c);
+  a = fma(-two_pi, rint(a * inv_two_pi), a);
+  __sincosf(static_cast<float>(a), s, c);
 }
 
 __global__ void rope_kernel(__nv_bfloat16 *__restrict__ x, int64_t m, int H, int d,
@@ -143,12 +144,17 @@ spts_status launch_gather_rows(const void *src, int64_t n_src, const int32_t *ro
 
 // ---------------------------------------------------------------- salience
 // Synthetic-workload step (not SPTS): K[rows[t], g] += shift * unit(mean of
-// the group's probe queries).  One block per KV head, d threads.
+// the group's probe queries).  Blocks (KV head, chunk of SAL_ROWS rows), d
+// threads; each block recomputes the group mean (a few KB of reads).
+constexpr int SAL_ROWS = 16;
+
 __global__ void inject_salience_kernel(__nv_bfloat16 *__restrict__ k, int64_t Nc, const __nv_bfloat16 *__restrict__ q,
                                        int P, int Hq, int Hkv, int d, const int32_t *__restrict__ rows, int64_t n_rows,
                                        float shift, uint32_t *status) {
   extern __shared__ float red[];
   const int g = blockIdx.x, i = threadIdx.x, G = Hq / Hkv;
+  const int64_t t_begin = static_cast<int64_t>(blockIdx.y) * SAL_ROWS;
+  const int64_t t_end = t_begin + SAL_ROWS < n_rows ? t_begin + SAL_ROWS : n_rows;
   double acc = 0.0;
   for (int p = 0; p < P; ++p)
     for (int j = 0; j < G; ++j) acc += __bfloat162float(q[(static_cast<int64_t>(p) * Hq + g * G + j) * d + i]);
@@ -160,7 +166,7 @@ __global__ void inject_salience_kernel(__nv_bfloat16 *__restrict__ k, int64_t Nc
     __syncthreads();
   }
   const float u = mean / sqrtf(red[0]);
-  for (int64_t t = 0; t < n_rows; ++t) {
+  for (int64_t t = t_begin; t < t_end; ++t) {
     const int32_t row = rows[t];
     if (row < 0 || row >= Nc) {
       if (i == 0) raise_status(status, SPTS_DEV_BADINDEX, 0x62u, static_cast<uint32_t>(row));
@@ -175,7 +181,8 @@ spts_status launch_inject_salience(void *k, int64_t Nc, const void *q_probe, int
                                    const int32_t *rows, int64_t n_rows, float shift, uint32_t *status,
                                    cudaStream_t s) {
   if (n_rows == 0) return SPTS_OK;
-  inject_salience_kernel<<<Hkv, d, d * sizeof(float), s>>>(static_cast<__nv_bfloat16 *>(k), Nc,
+  const dim3 grid(static_cast<unsigned>(Hkv), static_cast<unsigned>((n_rows + SAL_ROWS - 1) / SAL_ROWS));
+  inject_salience_kernel<<<grid, d, d * sizeof(float), s>>>(static_cast<__nv_bfloat16 *>(k), Nc,
                                                            static_cast<const __nv_bfloat16 *>(q_probe), P, Hq,
                                                            Hkv, d, rows, n_rows, shift, status);
   note_launch();
