@@ -166,19 +166,12 @@ class LayerCase:
                                  salient_shift=wl.salient_shift)
 
 
-def run_msdp_step(S, wl, h, pos, layers, f_buf):
-    """The MSDP pipeline: stages of two layers, pruning at each boundary."""
-    N = wl.N
-    li = 0
-    for ratio in wl.ratios:
-        k_s = keep_rows(ratio, N)
-        Nc = h.shape[0]
-        for _ in range(2):
-            desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, k_s, fuse=wl.fuse)
-            S.spts_layer_forward(h, pos, desc, layers[li], outputs={"f": f_buf[:Nc]})
-            li += 1
-        h, pos, _ = S.spts_stage_prune(f_buf[:Nc], k_s, wl.P, h, pos)
-    return h, pos
+def run_msdp_step(S, wl, h, pos, layers, desc):
+    """The MSDP pipeline (stages of two layers, pruning at each boundary) in
+    one C-ABI call; h and pos are compacted in place."""
+    ks = [keep_rows(r, wl.N) for r in wl.ratios]
+    S.spts_msdp_forward(h, pos, desc, layers, 2, ks)
+    return h
 
 
 def gpu_arm(args, rank, world, dev):
@@ -190,14 +183,14 @@ def gpu_arm(args, rank, world, dev):
     msdp = bool(wl.ratios)
     if msdp:
         base = LayerCase(S, wl, dev, 0)
-        layer_ws = [S.layer_weights({n: t.to(dev) for n, t in make_layer_weights(wl, i).items()})
-                    for i in range(wl.layers)]
-        keep_alive = [base]
-        layer_ws_refs = layer_ws
-        f_buf = torch.empty(wl.N, dtype=torch.float32, device=dev)
+        layer_tensors = [{n: t.to(dev) for n, t in make_layer_weights(wl, i).items()} for i in range(wl.layers)]
+        keep_alive = [base, layer_tensors]
+        mdesc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, 0, fuse=wl.fuse)
+        pos_buf = torch.empty_like(base.pos)
 
         def step(h):
-            return run_msdp_step(S, wl, h, base.pos, layer_ws_refs, f_buf)[0]
+            pos_buf.copy_(base.pos)        # the pipeline compacts positions in place
+            return run_msdp_step(S, wl, h, pos_buf, layer_tensors, mdesc)
     else:
         case = LayerCase(S, wl, dev)
         desc = case.desc()
@@ -261,7 +254,17 @@ def gpu_arm(args, rank, world, dev):
     dom_ms = by_name[dom]
     achieved = fl[dom] / (dom_ms / 1e3) / 1e12
     layer_flops = sum(fl.values())
-    layer_ms = float(stage_ms.sum())
+    if msdp:
+        # average layer of the pipeline: each stage's two layers at (|C_s|, k_s); the
+        # selected rows of later stages are taken as evenly spread over C_s
+        tot_f, tot_b, Nc = 0.0, 0.0, wl.N
+        for r_ in wl.ratios:
+            k_s = keep_rows(r_, wl.N)
+            f_s, b_s = layer_work(wl, Nc, k_s, wl.P, np.linspace(0, Nc - 1, k_s).astype(np.int64), ffn)
+            tot_f += 2 * sum(f_s.values())
+            tot_b += 2 * b_s
+            Nc = k_s
+        layer_flops, nbytes = tot_f / wl.layers, tot_b / wl.layers
     t_roof_ms = max(layer_flops / (peaks["bf16_sustained"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
 
     # ---------------- skipped-prefill speedup over the same kernels at keep 1.0

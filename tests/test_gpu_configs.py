@@ -23,6 +23,10 @@ if torch.cuda.is_available():
     import token_skipping_sparse_b200 as S
 
 
+PER_CALL_TOL = 2e-2     # bf16 outputs of one call given the same inputs
+LAYER_OUT_TOL = 4e-2    # the layer output: two bf16-stored stages composed
+
+
 def _f64(t):
     return t.float().double().numpy()
 
@@ -137,7 +141,10 @@ def _check_layer_sampled(wl, h, W, pos, sal, g, k, n_rows=40):
     ho = g["h_out"].numpy()
     fsel = rr[np.isin(rr, idf)]
     want = O.reduced_ffn(h1, np.where(np.isin(rr, idf))[0], None, 1e-5, Wn["w_gate"], Wn["w_up"], Wn["w_down"])
-    assert_close(ho[rr], want, 2e-2, "h out (sampled rows)")
+    # The layer output crosses two bf16-stored stages computed independently on
+    # each side (O_sel, then the FFN input and activation), so one-ulp rounding
+    # flips of the first stage reach the second: twice the per-call bound.
+    assert_close(ho[rr], want, LAYER_OUT_TOL, "h out (sampled rows)")
     skip = np.setdiff1d(np.arange(N), idf)
     assert np.array_equal(ho[skip], ha[skip]), "rows skipped by the FFN changed"
     assert len(fsel) > 0
@@ -152,6 +159,28 @@ def test_layer_full_size_sampled(name):
     sal = salient_rows(wl.N, wl.P, wl.salient_frac, wl.seed)
     g = _run_gpu_layer(wl, h, W, pos, sal)
     _check_layer_sampled(wl, h, W, pos, sal, g, wl.k)
+
+
+@pytest.mark.parametrize("name", ["layer_32k", "layer_128k"])
+def test_reduced_ffn_full_size_sampled(name):
+    """spts_reduced_ffn alone at the full sizes, on synthetic inputs."""
+    wl = WORKLOADS[name]
+    rng = np.random.default_rng(1)
+    h = make_hidden(wl)
+    W = make_layer_weights(wl)
+    idx = np.sort(rng.choice(wl.N, wl.k, replace=False)).astype(np.int32)
+    hd = h.cuda()
+    S.spts_reduced_ffn(hd, torch.from_numpy(idx).cuda(), None, 1e-5, W["w_gate"].cuda(), W["w_up"].cuda(),
+                       W["w_down"].cuda())
+    S.check_device_status()
+    got = hd.cpu().numpy()
+    skip = np.setdiff1d(np.arange(wl.N), idx)
+    assert np.array_equal(got[skip], h.numpy()[skip]), "rows outside idx changed"
+    rows = idx[np.unique(np.concatenate([[0, len(idx) - 1], rng.choice(len(idx), 64, replace=False)]))]
+    Wn = {n: _f64(W[n]) for n in ("w_gate", "w_up", "w_down")}
+    want = O.reduced_ffn(h.numpy()[rows].astype(np.float64), np.arange(len(rows)), None, 1e-5, Wn["w_gate"],
+                         Wn["w_up"], Wn["w_down"])
+    assert_close(got[rows], want, PER_CALL_TOL, "reduced ffn rows")
 
 
 def _msdp_gpu(wl, h, layers_cpu):
@@ -209,4 +238,5 @@ def test_msdp_small_chain_matches_oracle():
             return   # the chains diverge legitimately from here on
         cand = want_pos
     assert np.array_equal(pos_out.numpy(), opos)
-    assert_close(h_out.numpy(), oh, 5e-2, "msdp final hidden states")
+    # eight layers of independently rounded stages on each side
+    assert_close(h_out.numpy(), oh, 4 * LAYER_OUT_TOL, "msdp final hidden states")

@@ -81,7 +81,8 @@ spts_status spts_ltp_scores(spts_dtype dt, const void *x, int64_t Nc, int D, con
                             int Dout, float *scores, void *ws, size_t ws_bytes, spts_stream stream) {
   const char *who = "spts_ltp_scores";
   SPTS_REQUIRE(dt == SPTS_BF16, SPTS_ERR_UNSUPPORTED, "%s: only bf16 is supported", who);
-  SPTS_REQUIRE(x && A && B && scores, SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(Nc == 0 || (x && scores), SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(A && B, SPTS_ERR_INVALID, "%s: NULL weights", who);
   SPTS_REQUIRE(Nc >= 0 && D > 0 && D % 64 == 0 && r >= 64 && r <= 256 && r % 64 == 0 && Dout > 0 &&
                    Dout % 256 == 0,
                SPTS_ERR_SHAPE, "%s: need D%%64==0, r in {64..256} step 64, Dout%%256==0 (D=%d r=%d Dout=%d)",
@@ -102,7 +103,7 @@ spts_status spts_select_topk(const float *s_a, const float *s_b, spts_fuse mode,
   const char *who = "spts_select_topk";
   SPTS_REQUIRE(mode == SPTS_FUSE_NONE || mode == SPTS_FUSE_MAXNORM_ADD || mode == SPTS_FUSE_MULTIPLY,
                SPTS_ERR_INVALID, "%s: unknown fusion mode %d", who, static_cast<int>(mode));
-  SPTS_REQUIRE(s_a && idx_out && (mode == SPTS_FUSE_NONE || s_b), SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(Nc == 0 || (s_a && idx_out && (mode == SPTS_FUSE_NONE || s_b)), SPTS_ERR_INVALID, "%s: NULL argument", who);
   SPTS_REQUIRE(0 <= force_tail && force_tail <= k && k <= Nc && Nc < (int64_t(1) << 31), SPTS_ERR_SHAPE,
                "%s: need 0 <= force_tail <= k <= Nc < 2^31 (tail=%lld k=%lld Nc=%lld)", who,
                static_cast<long long>(force_tail), static_cast<long long>(k), static_cast<long long>(Nc));
@@ -154,7 +155,7 @@ spts_status spts_reduced_ffn(spts_dtype dt, float *h, int64_t Nc, int D, const i
                              const void *w_down, int F, void *ws, size_t ws_bytes, spts_stream stream) {
   const char *who = "spts_reduced_ffn";
   SPTS_REQUIRE(dt == SPTS_BF16, SPTS_ERR_UNSUPPORTED, "%s: only bf16 weights are supported", who);
-  SPTS_REQUIRE(h && idx && w_gate && w_up && w_down, SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE((k == 0 || (h && idx)) && w_gate && w_up && w_down, SPTS_ERR_INVALID, "%s: NULL argument", who);
   SPTS_REQUIRE(k >= 0 && k <= Nc && D > 0 && D % 256 == 0 && F > 0 && F % 128 == 0, SPTS_ERR_SHAPE,
                "%s: need k <= Nc, D %% 256 == 0, F %% 128 == 0 (k=%lld Nc=%lld D=%d F=%d)", who,
                static_cast<long long>(k), static_cast<long long>(Nc), D, F);
@@ -208,7 +209,7 @@ spts_status spts_stage_prune(const float *scores, int64_t Nc, int64_t k_keep, in
 spts_status spts_rmsnorm_rows(const float *x, const int32_t *rows, int64_t m, int D, const void *w, float eps,
                               void *y, spts_stream stream) {
   const char *who = "spts_rmsnorm_rows";
-  SPTS_REQUIRE(x && y, SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(m == 0 || (x && y), SPTS_ERR_INVALID, "%s: NULL argument", who);
   SPTS_REQUIRE(m >= 0 && D > 0 && D % 8 == 0, SPTS_ERR_SHAPE, "%s: need D %% 8 == 0", who);
   SPTS_REQUIRE(aligned(x, 16) && aligned(y, 16) && (!w || aligned(w, 16)) && (!rows || aligned(rows, 4)),
                SPTS_ERR_INVALID, "%s: misaligned pointer", who);
@@ -217,7 +218,7 @@ spts_status spts_rmsnorm_rows(const float *x, const int32_t *rows, int64_t m, in
 
 spts_status spts_rope(void *x, int64_t m, int H, int d, const int32_t *pos, double theta, spts_stream stream) {
   const char *who = "spts_rope";
-  SPTS_REQUIRE(x && pos, SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(m == 0 || (x && pos), SPTS_ERR_INVALID, "%s: NULL argument", who);
   SPTS_REQUIRE(m >= 0 && H > 0 && d > 0 && d % 2 == 0 && d <= 256 && theta > 0, SPTS_ERR_SHAPE,
                "%s: need even d <= 256 and theta > 0", who);
   return launch_rope(x, m, H, d, pos, theta, cs(stream));
@@ -226,7 +227,7 @@ spts_status spts_rope(void *x, int64_t m, int H, int d, const int32_t *pos, doub
 spts_status spts_gather_rows(const void *src, int64_t n_src, const int32_t *rows, int64_t m, int64_t row_bytes,
                              void *dst, void *ws, spts_stream stream) {
   const char *who = "spts_gather_rows";
-  SPTS_REQUIRE(src && rows && dst, SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(m == 0 || (src && rows && dst), SPTS_ERR_INVALID, "%s: NULL argument", who);
   SPTS_REQUIRE(m >= 0 && n_src >= 0 && row_bytes > 0 && row_bytes % 16 == 0, SPTS_ERR_SHAPE,
                "%s: row_bytes must be a positive multiple of 16", who);
   SPTS_REQUIRE(aligned(src, 16) && aligned(dst, 16) && aligned(rows, 4), SPTS_ERR_INVALID,
@@ -241,7 +242,7 @@ spts_status spts_linear(const void *A, int64_t M, int K, const void *W, const vo
                         void *out, const int32_t *rows, const int32_t *row_pos, double theta, void *ws,
                         size_t ws_bytes, spts_stream stream) {
   const char *who = "spts_linear";
-  SPTS_REQUIRE(A && W && out, SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(W && (M == 0 || (A && out)), SPTS_ERR_INVALID, "%s: NULL argument", who);
   SPTS_REQUIRE(epi >= SPTS_EPI_STORE && epi <= SPTS_EPI_SCATTER_ADD, SPTS_ERR_INVALID, "%s: bad epilogue", who);
   SPTS_REQUIRE(M >= 0 && M < (int64_t(1) << 31) && K > 0 && K % 64 == 0 && N > 0, SPTS_ERR_SHAPE,
                "%s: need K %% 64 == 0 (K=%d)", who, K);

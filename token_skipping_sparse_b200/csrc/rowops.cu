@@ -51,10 +51,79 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const float *__restri
   }
 }
 
+// Single-pass variant for D = 256 * V8: each lane keeps its V8 pairs of
+// float4 in registers, so the row is read from memory once.
+template <int V8>
+__global__ void __launch_bounds__(256) rmsnorm_rows_reg_kernel(const float *__restrict__ x,
+                                                               const int32_t *__restrict__ rows, int64_t m,
+                                                               const __nv_bfloat16 *__restrict__ w, float eps,
+                                                               __nv_bfloat16 *__restrict__ y) {
+  constexpr int D = 256 * V8;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (i >= m) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t src = rows ? rows[i] : i;
+  const float4 *xr = reinterpret_cast<const float4 *>(x + src * D);
+  float4 a[V8], b[V8];
+#pragma unroll
+  for (int t = 0; t < V8; ++t) {
+    const int c = lane + 32 * t;  // 8-element column group
+    a[t] = __ldg(xr + 2 * c);
+    b[t] = __ldg(xr + 2 * c + 1);
+  }
+  float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int t = 0; t < V8; ++t) {
+    ss[0] += a[t].x * a[t].x + b[t].x * b[t].x;
+    ss[1] += a[t].y * a[t].y + b[t].y * b[t].y;
+    ss[2] += a[t].z * a[t].z + b[t].z * b[t].z;
+    ss[3] += a[t].w * a[t].w + b[t].w * b[t].w;
+  }
+  float s = (ss[0] + ss[1]) + (ss[2] + ss[3]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float inv = 1.0f / sqrtf(s / static_cast<float>(D) + eps);
+  uint4 *yr = reinterpret_cast<uint4 *>(y + i * D);
+#pragma unroll
+  for (int t = 0; t < V8; ++t) {
+    const int c = lane + 32 * t;
+    float v[8] = {a[t].x, a[t].y, a[t].z, a[t].w, b[t].x, b[t].y, b[t].z, b[t].w};
+    if (w) {
+      uint4 wv = __ldg(reinterpret_cast<const uint4 *>(w) + c);
+      const __nv_bfloat16 *wb = reinterpret_cast<const __nv_bfloat16 *>(&wv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = v[e] * inv * __bfloat162float(wb[e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = v[e] * inv;
+    }
+    uint4 o;
+    o.x = pack_bf16x2(v[0], v[1]);
+    o.y = pack_bf16x2(v[2], v[3]);
+    o.z = pack_bf16x2(v[4], v[5]);
+    o.w = pack_bf16x2(v[6], v[7]);
+    yr[c] = o;
+  }
+}
+
 spts_status launch_rmsnorm_rows(const float *x, const int32_t *rows, int64_t m, int D, const void *w, float eps,
                                 void *y, cudaStream_t s) {
   if (m == 0) return SPTS_OK;
   const int64_t blocks = (m + 7) / 8;
+  const __nv_bfloat16 *wb = static_cast<const __nv_bfloat16 *>(w);
+  __nv_bfloat16 *yb = static_cast<__nv_bfloat16 *>(y);
+  if (D == 4096) {
+    rmsnorm_rows_reg_kernel<16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, rows, m, wb, eps, yb);
+    note_launch();
+    SPTS_CUDA_TRY(cudaGetLastError());
+    return SPTS_OK;
+  }
+  if (D == 1024) {
+    rmsnorm_rows_reg_kernel<4><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, rows, m, wb, eps, yb);
+    note_launch();
+    SPTS_CUDA_TRY(cudaGetLastError());
+    return SPTS_OK;
+  }
   rmsnorm_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
       x, rows, m, D, static_cast<const __nv_bfloat16 *>(w), eps, static_cast<__nv_bfloat16 *>(y));
   note_launch();
