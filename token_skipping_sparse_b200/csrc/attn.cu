@@ -2,25 +2,27 @@
 // informative tokens attend to every candidate key, causally by original
 // position).
 //
-// One CTA per (Q tile, KV head).  A Q tile packs 128/G selected tokens x the
-// G query heads that share KV head g (G = Hq/Hkv), so every K/V tile loaded
-// serves all G heads in one M=128 MMA.
-//   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys into a
-//               3-stage ring (128-byte swizzle);
-//   warp 1      MMA: S = Q K^T into one of two TMEM buffers (M=128, N=128,
-//               K=128), then O += P V with P read from TMEM (the softmax
-//               writes it over the S values it consumed) and V an MN-major
-//               shared-memory operand, into a third TMEM region;
-//   warps 2..5  softmax, one thread per Q row: tcgen05.ld of its S row,
-//               causal mask (only on tiles that cross the diagonal), row max
-//               with independent accumulators, lazy rescaling of O in TMEM
-//               (only when the running max grows by more than 2^8), exp2 with
-//               the scale folded into one FFMA, bf16 P stored back to TMEM
-//               with tcgen05.st; at the end O / l -> bf16.
-// Keeping P in TMEM takes it off the shared-memory path: per key tile the
-// shared memory then serves only the K and V tiles (TMA in, MMA out).
-// The key loop stops at the last key visible to the tile's latest query, and
-// tiles are launched latest-first so the long ones start early.
+// One CTA per (pair of Q tiles, KV head).  A Q tile packs 128/G selected
+// tokens x the G query heads that share KV head g (G = Hq/Hkv); a CTA holds
+// two consecutive Q tiles, A and B, so every K/V tile it loads feeds four
+// M=128 MMAs (S and PV for each tile) and the softmax of one tile runs while
+// the tensor core works on the other.
+//   warp 0      TMA: both Q tiles once, then K and V tiles of 128 keys into
+//               a 2-stage ring (128-byte swizzle);
+//   warp 1      MMA, per key tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).
+//               S_X = Q_X K^T lands in TMEM region S_X; the softmax writes
+//               bf16 P over it and PV reads P from TMEM (A operand in TMEM)
+//               with V an MN-major shared-memory operand, into O_X.
+//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B, one thread
+//               per Q row: tcgen05.ld of the S row, causal mask (only on key
+//               tiles crossing the tile's diagonal), row max with independent
+//               three-input max accumulators, lazy O rescale (only when the
+//               running max grows by more than 2^8), the scale folded into a
+//               packed fp32x2 FFMA before exp2, row sums in packed fp32x2
+//               adds, bf16 P back to TMEM; at the end O / l -> bf16.
+// Tile A holds the earlier tokens, so its key range is a prefix of B's: the
+// MMA and the softmax of A stop at A's own last visible key.  Pairs are
+// launched latest-first so the long ones start early.
 // All barrier waits are bounded (see sm100.cuh).
 #include <climits>
 
@@ -31,24 +33,24 @@
 namespace spts {
 namespace {
 
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;
 constexpr int BKV = 128;
-constexpr int KV_STAGES = 3;
+constexpr int KV_STAGES = 2;
 constexpr int TILE_BYTES = 128 * 128 * 2;  // 32 KB: 128 rows x 128 bf16, as two 64-wide swizzled chunks
 constexpr int CHUNK_BYTES = 128 * 64 * 2;  // 16 KB
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + TILE_BYTES;               // KV_STAGES stages
+constexpr int OFF_Q = 0;                                // Q_A, Q_B
+constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;           // KV_STAGES stages
 constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;   // KV_STAGES stages
 constexpr int OFF_BAR = OFF_V + KV_STAGES * TILE_BYTES;
 constexpr size_t SMEM_BYTES = OFF_BAR + 256;
-constexpr uint32_t TMEM_COLS = 512;  // S/P buffers [0,128) and [128,256), O [256,384)
+constexpr uint32_t TMEM_COLS = 512;  // S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
 struct Params {
   const int32_t *qpos;
   const int32_t *kpos;
   __nv_bfloat16 *o;
-  int m, Nc, Hq, Hkv, G, tq, n_qtiles;
+  int m, Nc, Hq, Hkv, G, tq, n_pairs;
   float scale_log2;
   uint32_t *status;
   uint64_t wait_ns;
@@ -58,6 +60,32 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pairs (sm_100a f32x2 arithmetic) and a three-input max: they
+// halve the instruction count of the softmax's per-element work.
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ int upper_bound(const int32_t *a, int n, int32_t v) {
@@ -79,17 +107,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t *sV = smem + OFF_V;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = k_full + KV_STAGES, *kv_empty = v_full + KV_STAGES,
-           *s_full = kv_empty + KV_STAGES, *p_ready = s_full + 2, *p_free = p_ready + 2, *drain = p_free + 2;
+           *s_full = kv_empty + KV_STAGES, *p_ready = s_full + 2, *o_done = p_ready + 2, *drain = o_done + 2;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-  int *s_range = reinterpret_cast<int *>(tmem_holder + 2);  // kv_end, mask_from
+  int *s_range = reinterpret_cast<int *>(tmem_holder + 2);  // per tile X: kv_end[X], mask_from[X]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / p.Hkv;
+  const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / p.Hkv;
   const int g = static_cast<int>(blockIdx.x) % p.Hkv;
-  const int t0 = qt * p.tq;
+  const int t0 = pair * 2 * p.tq;  // first token of tile A; tile B starts at t0 + tq
 
-  // The swizzled operand layouts need a 1024-byte aligned base.
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) raise_status(p.status, SPTS_DEV_BADINDEX, 0x2Fu, smem_u32(smem));
     return;
@@ -101,17 +128,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_ready[s], 128);
-      mbar_init(&p_free[s], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_ready[x], 128);
+      mbar_init(&o_done[x], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    const int last = min(t0 + p.tq, p.m) - 1;
-    s_range[0] = upper_bound(p.kpos, p.Nc, p.qpos[last]);
-    s_range[1] = upper_bound(p.kpos, p.Nc, p.qpos[t0]);
+    for (int x = 0; x < 2; ++x) {
+      const int first = t0 + x * p.tq;
+      if (first < p.m) {
+        const int last = min(first + p.tq, p.m) - 1;
+        s_range[2 * x] = upper_bound(p.kpos, p.Nc, p.qpos[last]);
+        s_range[2 * x + 1] = upper_bound(p.kpos, p.Nc, p.qpos[first]);
+      } else {
+        s_range[2 * x] = 0;  // tile B beyond the last token: no work
+        s_range[2 * x + 1] = 0;
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, TMEM_COLS);
@@ -121,20 +156,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int kv_end = s_range[0];
-  const int mask_from = s_range[1];
-  const int n_tiles = (kv_end + BKV - 1) / BKV;
+  const int n_a = (s_range[0] + BKV - 1) / BKV;
+  const int n_b = (s_range[2] + BKV - 1) / BKV;
+  const int n_kv = max(n_a, n_b);
 
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, TILE_BYTES);
-      tma_load_3d(sQ, &tmQ, q_full, 0, g * p.G, t0);
-      tma_load_3d(sQ + CHUNK_BYTES, &tmQ, q_full, 64, g * p.G, t0);
+      mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
+      for (int x = 0; x < 2; ++x) {
+        tma_load_3d(sQ + x * TILE_BYTES, &tmQ, q_full, 0, g * p.G, t0 + x * p.tq);
+        tma_load_3d(sQ + x * TILE_BYTES + CHUNK_BYTES, &tmQ, q_full, 64, g * p.G, t0 + x * p.tq);
+      }
       uint32_t issued = 0, issued_par = 0;
-      for (int j = 0; j < n_tiles; ++j) {
+      for (int j = 0; j < n_kv; ++j) {
         const int st = j % KV_STAGES;
         const uint32_t ph = (j / KV_STAGES) & 1;
         if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_flag, p.status, p.wait_ns, 0x21u)) break;
@@ -163,58 +200,70 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status, p.wait_ns, 0x22u);
       tc_fence_after();
-      const uint32_t q_addr = smem_u32(sQ);
-      // S_j goes to TMEM buffer j % 2.  tcgen05.mma from this thread run in
-      // issue order, so S_{j+2} (issued after PV_j) cannot overwrite P_j
-      // before PV_j has read it.
-      auto issue_s = [&](int j) -> bool {
+      // S_X(j) into TMEM region S_X.  tcgen05.mma from this thread run in
+      // issue order, so S_X(j+1) (issued after PV_X(j)) cannot overwrite P_X(j)
+      // before PV_X(j) has read it.
+      auto issue_s = [&](int x, int j) -> bool {
         const int st = j % KV_STAGES;
         if (!mbar_wait(&k_full[st], (j / KV_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x23u)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(sK + st * TILE_BYTES);
+        const uint32_t q_addr = smem_u32(sQ + x * TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t a = sdesc_k_sw128(q_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3);
           const uint64_t b = sdesc_k_sw128(k_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3);
-          mma_bf16_ss(tmem + (j & 1) * BKV, a, b, idesc_s, kk > 0);
+          mma_bf16_ss(tmem + x * BKV, a, b, idesc_s, kk > 0);
         }
-        tc_commit(&s_full[j & 1]);
+        tc_commit(&s_full[x]);
         return true;
       };
-      if (ok && n_tiles > 0) ok = issue_s(0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles && !issue_s(j + 1)) break;
-        const int b = j & 1, st = j % KV_STAGES;
-        if (!mbar_wait(&p_ready[b], (j >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x24u)) break;
-        if (!mbar_wait(&v_full[st], (j / KV_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x25u)) break;
+      auto issue_pv = [&](int x, int j) -> bool {
+        const int st = j % KV_STAGES;
+        if (!mbar_wait(&p_ready[x], j & 1, abort_flag, p.status, p.wait_ns, 0x24u)) return false;
+        if (!mbar_wait(&v_full[st], (j / KV_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x25u)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(sV + st * TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t v = sdesc_mn_sw128(v_addr + kk * 16 * 128, CHUNK_BYTES);
-          mma_bf16_ts(tmem + 256, tmem + b * BKV + kk * 8, v, idesc_pv, (j | kk) != 0);
+          mma_bf16_ts(tmem + 256 + x * 128, tmem + x * BKV + kk * 8, v, idesc_pv, (j | kk) != 0);
         }
-        tc_commit(&kv_empty[st]);
-        tc_commit(&p_free[b]);
+        tc_commit(&o_done[x]);
+        return true;
+      };
+      for (int x = 0; ok && x < 2; ++x)
+        if ((x == 0 ? n_a : n_b) > 0) ok = issue_s(x, 0);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        for (int x = 0; ok && x < 2; ++x) {
+          const int nxx = x == 0 ? n_a : n_b;
+          if (j >= nxx) continue;
+          ok = issue_pv(x, j);
+          if (ok && j + 1 < nxx) ok = issue_s(x, j + 1);
+        }
+        if (ok) tc_commit(&kv_empty[j % KV_STAGES]);  // both tiles are done with K/V tile j
       }
       tc_commit(drain);
       mbar_drain(drain, 0, p.status);
     }
     __syncwarp();
   } else {
-    // softmax warps: TMEM lane quadrant = warp % 4
+    // ---------------- softmax: warps 2..5 tile A, warps 6..9 tile B
+    const int x = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const int tok = t0 + r / p.G;
+    const int tok = t0 + x * p.tq + r / p.G;
     const bool valid = tok < p.m;
     const int32_t qp = valid ? p.qpos[tok] : INT_MIN;
+    const int kv_end = s_range[2 * x], mask_from = s_range[2 * x + 1];
+    const int n_tiles = x == 0 ? n_a : n_b;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t s_col = x * BKV, o_col = 256 + x * 128;
     const float c2 = p.scale_log2;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const int b = j & 1;
-      ok = mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x26u);
+      ok = mbar_wait(&s_full[x], j & 1, abort_flag, p.status, p.wait_ns, 0x26u);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -223,35 +272,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t xr[BKV];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        tmem_ld32(lane_base + b * BKV + c * 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32 * c));
+        tmem_ld32(lane_base + s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32 * c));
       tmem_ld_wait();
-      // raw scores; the scale (> 0) is folded into the row max and the exp2 FFMA
-      float x[BKV];
-#pragma unroll
-      for (int c = 0; c < BKV; ++c) x[c] = __uint_as_float(xr[c]);
       const int j0 = j * BKV;
       const bool need_mask = (j0 + BKV > mask_from) || (j0 + BKV > kv_end);
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < BKV; ++c) {
           const int key = j0 + c;
-          if (!(key < kv_end && __ldg(p.kpos + key) <= qp)) x[c] = -INFINITY;
+          if (!(key < kv_end && __ldg(p.kpos + key) <= qp)) xr[c] = 0xff800000u;  // -inf
         }
       }
       float m8[8];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) m8[t] = x[t];
+      for (int t = 0; t < 8; ++t) m8[t] = __uint_as_float(xr[t]);
 #pragma unroll
-      for (int c = 8; c < BKV; ++c) m8[c & 7] = fmaxf(m8[c & 7], x[c]);
+      for (int c = 8; c < BKV; c += 2)
+        m8[(c >> 1) & 7] = fmax3(m8[(c >> 1) & 7], __uint_as_float(xr[c]), __uint_as_float(xr[c + 1]));
       const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                              fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * c2;
       const float m_new = fmaxf(m_run, mt);
       const bool need = m_new > m_run + RESCALE_THRESHOLD;
       if (__any_sync(0xffffffffu, need)) {
         const float factor = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
-        if (j > 0) {
-          const int pb = (j - 1) & 1;
-          const bool okw = mbar_wait(&p_free[pb], ((j - 1) >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x27u);
+        if (j > 0) {  // O_X holds PV_X(0..j-1): wait for the last of them
+          const bool okw = mbar_wait(&o_done[x], (j - 1) & 1, abort_flag, p.status, p.wait_ns, 0x27u);
           if (!__all_sync(0xffffffffu, okw)) {
             ok = false;
             break;
@@ -260,11 +305,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
-            tmem_ld32(lane_base + 256 + c * 32, o);
+            tmem_ld32(lane_base + o_col + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
             for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * factor);
-            tmem_st32(lane_base + 256 + c * 32, o);
+            tmem_st32(lane_base + o_col + c * 32, o);
           }
           tmem_st_wait();
         }
@@ -272,30 +317,38 @@ __global__ void __launch_bounds__(THREADS, 1)
         m_run = m_new;
       }
       const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const uint64_t cc = f2pack(c2, c2), mm = f2pack(neg_m, neg_m);
+      uint64_t s4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          const float e0 = ex2(fmaf(x[h * 64 + 2 * t], c2, neg_m));
-          const float e1 = ex2(fmaf(x[h * 64 + 2 * t + 1], c2, neg_m));
-          s8[(2 * t) & 7] += e0;
-          s8[(2 * t + 1) & 7] += e1;
+          float a0, a1;
+          f2unpack(f2fma(f2pack(__uint_as_float(xr[h * 64 + 2 * t]), __uint_as_float(xr[h * 64 + 2 * t + 1])), cc,
+                         mm),
+                   a0, a1);
+          const float e0 = ex2(a0), e1 = ex2(a1);
+          s4[t & 3] = f2add(s4[t & 3], f2pack(e0, e1));
           pk[t] = pack_bf16x2(e0, e1);
         }
-        // P over the S values of this buffer: columns [b*128 + 32h, +32) hold keys [64h, 64h+64)
-        tmem_st32(lane_base + b * BKV + h * 32, pk);
+        // P over this tile's S values: columns [32h, 32h+32) hold keys [64h, 64h+64)
+        tmem_st32(lane_base + s_col + h * 32, pk);
       }
-      l += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+      {
+        float q0, q1, q2, q3, q4, q5, q6, q7;
+        f2unpack(f2add(s4[0], s4[1]), q0, q1);
+        f2unpack(f2add(s4[2], s4[3]), q2, q3);
+        (void)q4; (void)q5; (void)q6; (void)q7;
+        l += (q0 + q1) + (q2 + q3);
+      }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_ready[b]);
+      mbar_arrive(&p_ready[x]);
     }
-    // final normalisation once the last PV has landed
+    // final normalisation once the last PV of this tile has landed
     if (ok && n_tiles > 0) {
-      const int pb = (n_tiles - 1) & 1;
-      const bool okw = mbar_wait(&p_free[pb], ((n_tiles - 1) >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x29u);
+      const bool okw = mbar_wait(&o_done[x], (n_tiles - 1) & 1, abort_flag, p.status, p.wait_ns, 0x29u);
       ok = __all_sync(0xffffffffu, okw);
       if (ok) tc_fence_after();
     }
@@ -306,7 +359,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          tmem_ld32(lane_base + 256 + c * 32, o);
+          tmem_ld32(lane_base + o_col + c * 32, o);
           tmem_ld_wait();
           if (valid) {
             uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
@@ -369,13 +422,13 @@ spts_status launch_attention_bf16(const void *q, const int32_t *qpos, int64_t m,
   p.Hkv = Hkv;
   p.G = G;
   p.tq = tq;
-  p.n_qtiles = static_cast<int>((m + tq - 1) / tq);
+  p.n_pairs = static_cast<int>((m + 2 * tq - 1) / (2 * tq));
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = status;
   p.wait_ns = wait_limit_ns();
   SPTS_CUDA_TRY(cudaFuncSetAttribute(attention_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(SMEM_BYTES)));
-  const unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(Hkv);
+  const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(Hkv);
   attention_bf16_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tq_map, tk_map, tv_map, p);
   note_launch();
   SPTS_CUDA_TRY(cudaGetLastError());

@@ -39,6 +39,30 @@ void carve(Carver &cv, const spts_layer_desc *L, int64_t Nc, LayerBufs &b) {
   b.qpos = static_cast<int32_t *>(cv.take(k * 4));
 }
 
+// A side stream and fork/join events per (host thread, device): the V and
+// probe-Q projections run on it while the main stream does the K projection,
+// the probe scores, the selection and the gathers, which leave most SMs idle.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, qprobe_done = nullptr, v_done = nullptr;
+};
+
+spts_status side_stream(SideStream **out) {
+  static thread_local SideStream per_dev[64];
+  int dev = 0;
+  SPTS_CUDA_TRY(cudaGetDevice(&dev));
+  SPTS_REQUIRE(dev >= 0 && dev < 64, SPTS_ERR_UNSUPPORTED, "spts_layer_forward: device ordinal %d", dev);
+  SideStream &ss = per_dev[dev];
+  if (ss.s == nullptr) {
+    SPTS_CUDA_TRY(cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking));
+    SPTS_CUDA_TRY(cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming));
+    SPTS_CUDA_TRY(cudaEventCreateWithFlags(&ss.qprobe_done, cudaEventDisableTiming));
+    SPTS_CUDA_TRY(cudaEventCreateWithFlags(&ss.v_done, cudaEventDisableTiming));
+  }
+  *out = &ss;
+  return SPTS_OK;
+}
+
 spts_status check_layer(const spts_layer_desc *L, const spts_layer_weights *W, int64_t Nc) {
   const char *who = "spts_layer_forward";
   SPTS_REQUIRE(L && W, SPTS_ERR_INVALID, "%s: NULL descriptor", who);
@@ -102,19 +126,43 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
     return SPTS_OK;
   };
 
+  // Stage events time the stages one after another, so with them the side
+  // stream is not used and every kernel runs on the caller's stream.
+  SideStream *side = nullptr;
+  if (o.stage_events == nullptr) SPTS_TRY(side_stream(&side));
+  // On any early return after the fork, still order the caller's stream
+  // behind the side stream's work on the workspace.
+  struct JoinGuard {
+    SideStream *side;
+    cudaStream_t s;
+    bool joined;
+    ~JoinGuard() {
+      if (side && !joined) cudaStreamWaitEvent(s, side->v_done, 0);
+    }
+  } guard{side, s, false};
+
   // a1-a2: norm, K (+RoPE) / V for every candidate, Q (+RoPE) for the probe rows
   SPTS_TRY(mark(0));
   SPTS_TRY(launch_rmsnorm_rows(h, nullptr, Nc, D, W->norm_attn, L->eps, b.xn, s));
   SPTS_TRY(mark(1));
+  const void *xtail = static_cast<const char *>(b.xn) + static_cast<size_t>(Nc - P) * D * 2;
+  GemmArgs gq{xtail, P, D, W->w_q, nullptr, hq, SPTS_EPI_ROPE, b.qprobe, nullptr, pos + (Nc - P), L->theta, st};
+  GemmArgs gv{b.xn, Nc, D, W->w_v, nullptr, hk, SPTS_EPI_STORE, b.vv, nullptr, nullptr, 0.0, st};
+  if (side) {  // fork: probe-Q and V projections on the side stream
+    SPTS_CUDA_TRY(cudaEventRecord(side->fork, s));
+    SPTS_CUDA_TRY(cudaStreamWaitEvent(side->s, side->fork, 0));
+    SPTS_TRY(launch_gemm(gq, side->s));
+    SPTS_CUDA_TRY(cudaEventRecord(side->qprobe_done, side->s));
+    SPTS_TRY(launch_gemm(gv, side->s));
+    SPTS_CUDA_TRY(cudaEventRecord(side->v_done, side->s));
+  }
   GemmArgs gk{b.xn, Nc, D, W->w_k, nullptr, hk, SPTS_EPI_ROPE, b.kk, nullptr, pos, L->theta, st};
   SPTS_TRY(launch_gemm(gk, s));
   SPTS_TRY(mark(2));
-  GemmArgs gv{b.xn, Nc, D, W->w_v, nullptr, hk, SPTS_EPI_STORE, b.vv, nullptr, nullptr, 0.0, st};
-  SPTS_TRY(launch_gemm(gv, s));
+  if (!side) SPTS_TRY(launch_gemm(gv, s));
   SPTS_TRY(mark(3));
-  const void *xtail = static_cast<const char *>(b.xn) + static_cast<size_t>(Nc - P) * D * 2;
-  GemmArgs gq{xtail, P, D, W->w_q, nullptr, hq, SPTS_EPI_ROPE, b.qprobe, nullptr, pos + (Nc - P), L->theta, st};
-  SPTS_TRY(launch_gemm(gq, s));
+  if (side) SPTS_CUDA_TRY(cudaStreamWaitEvent(s, side->qprobe_done, 0));
+  else SPTS_TRY(launch_gemm(gq, s));
   if (L->n_salient > 0)
     SPTS_TRY(launch_inject_salience(b.kk, Nc, b.qprobe, P, L->Hq, L->Hkv, L->d, L->salient_rows, L->n_salient,
                                     L->salient_shift, st, s));
@@ -135,6 +183,10 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   GemmArgs gqs{b.xsel, k, D, W->w_q, nullptr, hq, SPTS_EPI_ROPE, b.qsel, nullptr, b.qpos, L->theta, st};
   SPTS_TRY(launch_gemm(gqs, s));
   SPTS_TRY(mark(8));
+  if (side) {  // join: V is ready
+    SPTS_CUDA_TRY(cudaStreamWaitEvent(s, side->v_done, 0));
+    guard.joined = true;
+  }
   SPTS_TRY(launch_attention_bf16(b.qsel, b.qpos, k, b.kk, b.vv, pos, Nc, L->Hq, L->Hkv, scale, osel, st, s));
   SPTS_TRY(mark(9));
   GemmArgs go{osel, k, hq, W->w_o, nullptr, D, SPTS_EPI_SCATTER_ADD, h, idx_a, nullptr, 0.0, st};

@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-// merge the splits: stats[g][row] = (max, 1/sum) in log2 units
+// merge the splits: stats[g][row].x = max + log2(sum) in log2 units
 __global__ void probe_combine_kernel(const float2 *__restrict__ partial, int splits, int total,
                                      float2 *__restrict__ stats) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -235,7 +235,8 @@ __global__ void probe_combine_kernel(const float2 *__restrict__ partial, int spl
       const float2 v = partial[static_cast<int64_t>(s) * total + i];
       if (v.x != -INFINITY) l += v.y * ex2(v.x - m);
     }
-  stats[i] = make_float2(m == -INFINITY ? 0.f : m, l > 0.f ? 1.f / l : 0.f);
+  // pass 2 weighs key j by 2^(s_j - m - log2 l): fold the normaliser into the exponent
+  stats[i] = make_float2(l > 0.f ? m + __log2f(l) : INFINITY, 0.f);
 }
 
 // ------------------------------------------------------------------ pass 2
@@ -252,8 +253,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int q_tiles = ncol / 128;
   uint8_t *sQ = smem;                          // q_tiles x 32 KB: rows [ncol] as 64-wide chunks per tile
   uint8_t *sK = smem + q_tiles * TILE_BYTES;   // P2_STAGES x 32 KB
-  float2 *sstat = reinterpret_cast<float2 *>(sK + P2_STAGES * TILE_BYTES);
-  int32_t *scol = reinterpret_cast<int32_t *>(sstat + P2_MAX_ROWS);
+  float *smm = reinterpret_cast<float *>(sK + P2_STAGES * TILE_BYTES);   // per column: max + log2(sum)
+  int32_t *scol = reinterpret_cast<int32_t *>(smm + P2_MAX_ROWS);      // per column: probe position
   uint64_t *bars = reinterpret_cast<uint64_t *>(scol + P2_MAX_ROWS);
   uint64_t *q_full = bars, *k_full = bars + 1, *k_empty = bars + 1 + P2_STAGES, *s_full = bars + 1 + 2 * P2_STAGES,
            *s_free = s_full + 2, *drain = s_free + 2;
@@ -264,13 +265,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x % chunks;
   const int g = blockIdx.x / chunks;
-  const int nbuf = (2 * ncol <= 512) ? 2 : 1;
+  // the probe rows are processed in chunks of CW columns, one TMEM buffer each
+  const int CW = (ncol % 256 == 0) ? 256 : 128;
+  const int nch = ncol / CW;
   const uint32_t tmem_cols = 512;
 
   for (int c = threadIdx.x; c < P2_MAX_ROWS; c += THREADS) {
     const int pr = c / p.G;
     const bool live = c < ncol && pr < p.P;
-    sstat[c] = live ? stats[g * ncol + c] : make_float2(0.f, 0.f);
+    smm[c] = live ? stats[g * ncol + c].x : INFINITY;
     scol[c] = live ? p.ppos[pr] : INT_MIN;
   }
   if (threadIdx.x == 0) {
@@ -335,29 +338,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const int nmma = ncol > 256 ? 2 : 1;
-      const int nper = ncol / nmma;  // 128 or 256 columns per MMA
-      const uint32_t idesc = idesc_bf16_f32(128, nper, 0, 0);
+      const uint32_t idesc = idesc_bf16_f32(128, CW, 0, 0);
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status, p.wait_ns, 0x42u);
       tc_fence_after();
-      for (int i = 0; ok && i < n; ++i) {
+      // work item it = (key tile it / nch, column chunk it % nch) into TMEM buffer it % 2
+      for (int it = 0; ok && it < n * nch; ++it) {
+        const int i = it / nch, h = it % nch;
         const int st = i % P2_STAGES;
-        const int b = nbuf == 2 ? (i & 1) : 0;
-        const uint32_t bpar = nbuf == 2 ? ((i >> 1) & 1) : (i & 1);
-        if (!mbar_wait(&s_free[b], bpar ^ 1u, abort_flag, p.status, p.wait_ns, 0x43u)) break;
-        if (!mbar_wait(&k_full[st], (i / P2_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x44u)) break;
+        const int b = it & 1;
+        if (!mbar_wait(&s_free[b], ((it >> 1) & 1) ^ 1u, abort_flag, p.status, p.wait_ns, 0x43u)) break;
+        if (h == 0 && !mbar_wait(&k_full[st], (i / P2_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x44u)) break;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(sK + st * TILE_BYTES);
-        for (int h = 0; h < nmma; ++h) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = sdesc_k_sw128(k_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3);
-            const uint32_t q_addr = smem_u32(sQ + (kk >> 2) * q_tiles * CHUNK_BYTES + h * (nper / 128) * CHUNK_BYTES);
-            const uint64_t bq = sdesc_k_sw128(q_addr) + 2 * (kk & 3);
-            mma_bf16_ss(tmem + b * ncol + h * nper, a, bq, idesc, kk > 0);
-          }
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sdesc_k_sw128(k_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3);
+          const uint32_t q_addr = smem_u32(sQ + (kk >> 2) * q_tiles * CHUNK_BYTES + h * (CW / 128) * CHUNK_BYTES);
+          mma_bf16_ss(tmem + b * CW, a, sdesc_k_sw128(q_addr) + 2 * (kk & 3), idesc, kk > 0);
         }
-        tc_commit(&k_empty[st]);
+        if (h == nch - 1) tc_commit(&k_empty[st]);
         tc_commit(&s_full[b]);
       }
       tc_commit(drain);
@@ -368,10 +367,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quad = warp & 3;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     bool ok = true;
-    for (int i = 0; i < n; ++i) {
-      const int b = nbuf == 2 ? (i & 1) : 0;
-      const uint32_t bpar = nbuf == 2 ? ((i >> 1) & 1) : (i & 1);
-      ok = mbar_wait(&s_full[b], bpar, abort_flag, p.status, p.wait_ns, 0x45u);
+    float acc = 0.f;
+    for (int it = 0; it < n * nch; ++it) {
+      const int i = it / nch, h = it % nch;
+      const int b = it & 1;
+      ok = mbar_wait(&s_full[b], (it >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x45u);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -381,24 +381,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool live = j < kv_end;
       const int32_t kp = live ? __ldg(p.kpos + j) : INT_MAX;
       const bool all_vis = kp <= ppos_min;
+      if (h == 0) acc = 0.f;
       float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-      for (int c0 = 0; c0 < ncol; c0 += 32) {
+      for (int c0 = 0; c0 < CW; c0 += 32) {
         uint32_t xr[32];
-        tmem_ld32(lane_base + b * ncol + c0, xr);
+        tmem_ld32(lane_base + b * CW + c0, xr);
         tmem_ld_wait();
+        const float *mmc = smm + h * CW + c0;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const float2 st = sstat[c0 + t];
-          float w = ex2(fmaf(__uint_as_float(xr[t]), p.scale_log2, -st.x)) * st.y;
-          if (!all_vis && kp > scol[c0 + t]) w = 0.f;
-          a4[t & 3] += w;
+        for (int t = 0; t < 32; t += 4) {
+          const float4 mq = *reinterpret_cast<const float4 *>(mmc + t);
+          const float mv[4] = {mq.x, mq.y, mq.z, mq.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float w = ex2(fmaf(__uint_as_float(xr[t + e]), p.scale_log2, -mv[e]));
+            if (!all_vis && kp > scol[h * CW + c0 + t + e]) w = 0.f;
+            a4[e] += w;
+          }
         }
       }
-      const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      acc += (a4[0] + a4[1]) + (a4[2] + a4[3]);
       tc_fence_before();
       mbar_arrive(&s_free[b]);
-      if (live) group[static_cast<int64_t>(g) * p.Nc + j] = acc;
+      if (h == nch - 1 && live) group[static_cast<int64_t>(g) * p.Nc + j] = acc;
     }
     // keys beyond every probe position get no weight
     if (ok) {
