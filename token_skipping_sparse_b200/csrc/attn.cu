@@ -13,7 +13,8 @@
 //               S_X = Q_X K^T lands in TMEM region S_X; the softmax writes
 //               bf16 P over it and PV reads P from TMEM (A operand in TMEM)
 //               with V an MN-major shared-memory operand, into O_X.
-//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B, one thread
+//   warps 2..3  idle (they complete warpgroup 0 for the register split);
+//   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B, one thread
 //               per Q row: tcgen05.ld of the S row, causal mask (only on key
 //               tiles crossing the tile's diagonal), row max with independent
 //               three-input max accumulators, lazy O rescale (only when the
@@ -33,7 +34,10 @@
 namespace spts {
 namespace {
 
-constexpr int THREADS = 320;
+constexpr int THREADS = 384;
+// setmaxnreg split: each SMSP holds one warp of warpgroup 0 and one softmax
+// warp of each tile: 56 + 2 x 224 = 3 x 168, the launch allocation.
+constexpr int REG_LOW = 56, REG_HIGH = 224;
 constexpr int BKV = 128;
 constexpr int KV_STAGES = 2;
 constexpr int TILE_BYTES = 128 * 128 * 2;  // 32 KB: 128 rows x 128 bf16, as two 64-wide swizzled chunks
@@ -161,6 +165,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int n_kv = max(n_a, n_b);
 
   if (warp == 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -195,6 +200,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, BKV, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
@@ -247,9 +253,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_drain(drain, 0, p.status);
     }
     __syncwarp();
+  } else if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));  // idle
   } else {
-    // ---------------- softmax: warps 2..5 tile A, warps 6..9 tile B
-    const int x = (warp - 2) >> 2;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_HIGH));
+    // ---------------- softmax: warps 4..7 tile A, warps 8..11 tile B
+    const int x = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int tok = t0 + x * p.tq + r / p.G;
