@@ -30,6 +30,18 @@ def test_linear_store(M, K, N):
     assert_bf16_close(np64(out), want, 1e-4, "linear store")
 
 
+
+def test_linear_store_more_tiles_than_sm_pairs():
+    # 40 x 4 tiles of 256 x 256 over at most 74 resident CTA pairs: every pair
+    # runs several tiles through both TMEM accumulators; M is ragged.
+    M, K, N = 10200, 256, 1024
+    A = torch.randn(M, K).to(torch.bfloat16)
+    W = _w(N, K)
+    out = S.spts_linear(A.cuda(), W.cuda())
+    want = O.bf16_round(np64(A) @ np64(W).T)
+    assert_bf16_close(np64(out), want, 1e-4, "linear store, many tiles")
+
+
 def test_linear_rope():
     M, K, H = 333, 512, 4
     A = torch.randn(M, K).to(torch.bfloat16)
