@@ -174,6 +174,28 @@ def run_msdp_step(S, wl, h, pos, layers, desc):
     return h
 
 
+
+def captured_traffic(workload: str):
+    """DRAM bytes (read + write) per launch of the dominant kernel, from the
+    committed ncu summary of that kernel on this workload, or None when there
+    is no capture for it or the kernel source changed since the capture (the
+    summary records a sha256 prefix of the source file)."""
+    import hashlib
+    import re
+    summary = os.path.join(ROOT, "profiles", f"attention_bf16_{workload}.md")
+    src = os.path.join(ROOT, "token_skipping_sparse_b200", "csrc", "attn.cu")
+    if not (os.path.exists(summary) and os.path.exists(src)):
+        return None
+    text = open(summary).read()
+    sha = re.search(r"sha256 prefix\s*`([0-9a-f]{16})`", text)
+    dram = re.search(r"DRAM read / write per launch \| ([0-9.]+) MB / ([0-9.]+) MB", text)
+    if not (sha and dram):
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != sha.group(1):
+        return None
+    return round((float(dram.group(1)) + float(dram.group(2))) * 1e6)
+
+
 def gpu_arm(args, rank, world, dev):
     import token_skipping_sparse_b200 as S
 
@@ -320,7 +342,8 @@ def gpu_arm(args, rank, world, dev):
                    "l2": "inputs larger than L2 (no flush)", "input": "each step runs on the previous step's output"},
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": round(achieved / peaks["bf16_sustained"], 4), "traffic": None,
+                     "frac": round(achieved / peaks["bf16_sustained"], 4),
+                     "traffic": captured_traffic(wl.name) if dom == "reduced_attention" else None,
                      "peak_note": f"{peaks['source']} sustained bf16 (kernel timed inside a long step)"},
         "layer_roofline": {"flops": layer_flops, "hbm_bytes": nbytes, "t_roof_ms": round(t_roof_ms, 4),
                            "ms_measured": round(ms_step / layers_per_step, 4),
