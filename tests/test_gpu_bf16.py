@@ -37,7 +37,7 @@ def test_reduced_attention_bf16(Nc, k, Hq, Hkv):
 
 
 @pytest.mark.parametrize("Nc,P,Hq,Hkv", [(1000, 16, 8, 2), (3000, 64, 32, 8), (2000, 128, 32, 8), (300, 64, 8, 8),
-                                         (700, 20, 8, 4)])
+                                         (700, 20, 8, 4), (2500, 80, 32, 8), (130, 100, 32, 8)])
 def test_probe_scores_bf16(Nc, P, Hq, Hkv):
     pos = _positions(Nc)
     q = torch.randn(P, Hq, 128).to(torch.bfloat16)

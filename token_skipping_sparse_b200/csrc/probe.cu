@@ -2,19 +2,24 @@
 //
 // Score of key j: s_j = sum over heads h and probes p of the causal softmax
 // weight a[h,p,j].  Two passes over the keys, both on tcgen05:
-//   pass 1 (row statistics): per (KV head g, tile of 128 probe rows, key
-//     split) a CTA computes S = Q K^T for its key range (M = 128 rows =
-//     128/G probes x G heads, N = 128 keys) and keeps each row's running max
-//     and sum of exp2 (log2 domain).  A combine kernel merges the splits into
-//     (max, 1/sum) per row.
-//   pass 2 (column sums): per (KV head g, key chunk) a CTA holds all of the
-//     group's probe rows in shared memory and computes the transposed tile
-//     S^T = K Q^T (M = 128 keys, N = probe rows), so each TMEM lane is one
-//     key and its score is a per-thread sum over the row: no atomics, fixed
-//     order, deterministic.  It writes group_scores[g][j]; a final kernel
-//     adds the groups.
-// Warp roles as in the other kernels: warp 0 TMA, warp 1 MMA, warps 2..5
-// consume the accumulators.  All waits are bounded.
+//   pass 1 (row statistics): per (KV head g, key split) a CTA holds the Q
+//     tiles of all of the group's probe rows (up to 4 x 128 rows: 128/G
+//     probes x G heads each) and, for every key tile of its range, computes
+//     S = Q_u K^T for each row tile u (M = 128 rows, N = 128 keys), keeping
+//     each row's running max and sum of exp2 (log2 domain).  A combine kernel
+//     merges the partial statistics into max + log2(sum) per row.
+//   pass 2 (column sums): per (KV head g, key split) a CTA holds all of the
+//     group's probe rows and computes transposed tiles S^T = K Q_u^T (M = 128
+//     keys, N = 128 probe rows of chunk u), so each TMEM lane is one key and
+//     its score is a per-thread sum over the row: no atomics, fixed order,
+//     deterministic.  It writes group_scores[g][j]; a final kernel adds the
+//     groups.
+// Both passes: warp 0 TMA, warp 1 MMA, two consumer warpgroups (warps 4..7
+// and 8..11) that take alternate key tiles, each with two TMEM buffers of 128
+// columns, so that one warpgroup's exponentials overlap the other's and the
+// MMAs of the next work items.  A K tile is loaded once per CTA and feeds all
+// row tiles (pass 1) or column chunks (pass 2).  The grids are one wave: one
+// CTA per SM.  All waits are bounded.
 #include <climits>
 
 #include "host.hpp"
@@ -24,11 +29,17 @@
 namespace spts {
 namespace {
 
-constexpr int THREADS = 192;
+constexpr int THREADS = 384;
+// setmaxnreg split: per SMSP one warp of warpgroup 0 (TMA, MMA, idle) and
+// one warp of each consumer warpgroup: 80 + 2 x 208 <= 3 x 168.
+constexpr int REG_LOW = 80, REG_HIGH = 208;
 constexpr int BKEY = 128;
-constexpr int TILE_BYTES = 128 * 128 * 2;
+constexpr int TILE_BYTES = 128 * 128 * 2;  // 128 rows x 128 bf16 as two 64-wide swizzled chunks
 constexpr int CHUNK_BYTES = 128 * 64 * 2;
+constexpr int MAX_RT = 4;                  // probe rows per group <= 512
 constexpr int MAX_SPLITS = 64;
+constexpr int MAX_STAGES = 4;
+constexpr int SMEM_CAP = 232448;           // dynamic shared memory per CTA on sm_100
 constexpr float LOG2E = 1.4426950408889634f;
 
 __device__ __forceinline__ float ex2(float x) {
@@ -36,15 +47,36 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 
-__device__ __forceinline__ int upper_bound(const int32_t *a, int n, int32_t v) {
-  int lo = 0, hi = n;
+// Number of a[0..n) that are <= v (a sorted ascending), by the whole warp:
+// each step samples 32 evenly spaced points, so 2^17 keys take 4 dependent
+// loads instead of 17.
+__device__ __forceinline__ int warp_upper_bound(const int32_t *a, int n, int32_t v) {
+  const int lane = threadIdx.x & 31;
+  int lo = 0, hi = n;  // answer in [lo, hi]
   while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (a[mid] <= v) lo = mid + 1;
-    else hi = mid;
+    const int step = (hi - lo + 31) >> 5;
+    const int idx = lo + (lane + 1) * step - 1;
+    const bool le = idx < hi && __ldg(a + idx) <= v;
+    const int cnt = __popc(__ballot_sync(0xffffffffu, le));  // samples 0..cnt-1 are <= v
+    const int nlo = lo + cnt * step;
+    const int nhi = lo + (cnt + 1) * step - 1;
+    lo = nlo;
+    if (nhi < hi) hi = nhi;
   }
   return lo;
+}
+
+// Work item (local key tile i, sub-item u) uses TMEM buffer (i & 1) * 2 + (u & 1)
+// and consumer warpgroup i & 1.  Uses of that buffer before this item:
+__device__ __forceinline__ uint32_t buffer_uses(int i, int u, int nsub) {
+  const int per_tile = (nsub - (u & 1) + 1) >> 1;  // sub-items of u's parity per key tile
+  return static_cast<uint32_t>((i >> 1) * per_tile + (u >> 1));
 }
 
 struct Geo {
@@ -52,186 +84,295 @@ struct Geo {
   const int32_t *kpos;  // [Nc]
   int P, Nc, Hq, Hkv, G, tq;
   int rows_pad;         // probe rows per group padded to 128
+  int n_sub;            // row tiles (pass 1) / column chunks (pass 2) = rows_pad / 128
+  int splits;           // key splits (CTAs per group)
+  int stages;           // K ring depth
   float scale_log2;
   uint32_t *status;
   uint64_t wait_ns;
 };
 
-// ------------------------------------------------------------------ pass 1
-constexpr int P1_STAGES = 3;
-constexpr int P1_OFF_Q = 0;
-constexpr int P1_OFF_K = TILE_BYTES;
-constexpr int P1_OFF_BAR = P1_OFF_K + P1_STAGES * TILE_BYTES;
-constexpr size_t P1_SMEM = 1024 + P1_OFF_BAR + 256;
+struct Smem {
+  uint8_t *q, *k;
+  uint64_t *q_full, *k_full, *k_empty, *s_full, *s_free, *drain;
+  uint32_t *tmem_holder;
+  volatile int *abort_flag;
+  int *ranges;  // [0..MAX_RT) kv_end per row tile, [MAX_RT..2 MAX_RT) mask_from, [2 MAX_RT] kv_end of the group
+  float *colv;  // pass 2: per column max + log2(sum)
+  int32_t *colp;  // pass 2: per column probe position
+};
 
-__global__ void __launch_bounds__(THREADS, 1)
-    probe_stats_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ Geo p, int n_rt, int splits, float2 *__restrict__ partial) {
-  extern __shared__ uint8_t smem_raw[];
+__device__ __forceinline__ Smem carve_smem(uint8_t *smem_raw, const Geo &p, bool cols) {
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = smem + P1_OFF_Q;
-  uint8_t *sK = smem + P1_OFF_K;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + P1_OFF_BAR);
-  uint64_t *q_full = bars, *k_full = bars + 1, *k_empty = bars + 1 + P1_STAGES, *s_full = bars + 1 + 2 * P1_STAGES,
-           *s_free = s_full + 2, *drain = s_free + 2;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-  int *s_range = reinterpret_cast<int *>(tmem_holder + 2);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x % splits;
-  const int rt = (blockIdx.x / splits) % n_rt;
-  const int g = blockIdx.x / (splits * n_rt);
-  const int p0 = rt * p.tq;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < P1_STAGES; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 128);
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-    const int last = min(p0 + p.tq, p.P) - 1;
-    const int kv_end = upper_bound(p.kpos, p.Nc, p.ppos[last]);
-    const int n_kt = (kv_end + BKEY - 1) / BKEY;
-    const int per = (n_kt + splits - 1) / splits;
-    s_range[0] = min(n_kt, split * per);
-    s_range[1] = min(n_kt, (split + 1) * per);
-    s_range[2] = kv_end;
-    s_range[3] = upper_bound(p.kpos, p.Nc, p.ppos[p0]);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_holder, 256);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  const int kt0 = s_range[0], kt1 = s_range[1], kv_end = s_range[2], mask_from = s_range[3];
-  const int n = kt1 - kt0;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, TILE_BYTES);
-      tma_load_3d(sQ, &tmQ, q_full, 0, g * p.G, p0);
-      tma_load_3d(sQ + CHUNK_BYTES, &tmQ, q_full, 64, g * p.G, p0);
-      uint32_t issued = 0, par = 0;
-      for (int i = 0; i < n; ++i) {
-        const int st = i % P1_STAGES;
-        const uint32_t ph = (i / P1_STAGES) & 1;
-        if (!mbar_wait(&k_empty[st], ph ^ 1u, abort_flag, p.status, p.wait_ns, 0x31u)) break;
-        mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
-        const int key0 = (kt0 + i) * BKEY;
-        tma_load_3d(sK + st * TILE_BYTES, &tmK, &k_full[st], 0, g, key0);
-        tma_load_3d(sK + st * TILE_BYTES + CHUNK_BYTES, &tmK, &k_full[st], 64, g, key0);
-        issued |= 1u << st;
-        par = (par & ~(1u << st)) | (ph << st);
-      }
-      if (*abort_flag) {
-        mbar_drain(q_full, 0, p.status);
-        for (int st = 0; st < P1_STAGES; ++st)
-          if (issued & (1u << st)) mbar_drain(&k_full[st], (par >> st) & 1u, p.status);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, BKEY, 0, 0);
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status, p.wait_ns, 0x32u);
-      tc_fence_after();
-      const uint32_t q_addr = smem_u32(sQ);
-      for (int i = 0; ok && i < n; ++i) {
-        const int st = i % P1_STAGES, b = i & 1;
-        if (!mbar_wait(&s_free[b], ((i >> 1) & 1) ^ 1u, abort_flag, p.status, p.wait_ns, 0x33u)) break;
-        if (!mbar_wait(&k_full[st], (i / P1_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x34u)) break;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + st * TILE_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + b * BKEY, sdesc_k_sw128(q_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3),
-                      sdesc_k_sw128(k_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3), idesc, kk > 0);
-        tc_commit(&k_empty[st]);
-        tc_commit(&s_full[b]);
-      }
-      tc_commit(drain);
-      mbar_drain(drain, 0, p.status);
-    }
-    __syncwarp();
+  Smem s;
+  s.q = smem;
+  s.k = smem + p.n_sub * TILE_BYTES;
+  uint8_t *tail = s.k + p.stages * TILE_BYTES;
+  if (cols) {
+    s.colv = reinterpret_cast<float *>(tail);
+    s.colp = reinterpret_cast<int32_t *>(tail + MAX_RT * 128 * 4);
+    tail += MAX_RT * 128 * 8;
   } else {
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;
-    const int pr = p0 + r / p.G;
-    const bool valid = pr < p.P;
-    const int32_t qp = valid ? p.ppos[pr] : INT_MIN;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int i = 0; i < n; ++i) {
-      const int b = i & 1;
-      ok = mbar_wait(&s_full[b], (i >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x35u);
-      if (!__all_sync(0xffffffffu, ok)) {
+    s.colv = nullptr;
+    s.colp = nullptr;
+  }
+  uint64_t *bars = reinterpret_cast<uint64_t *>(tail);
+  s.q_full = bars;
+  s.k_full = bars + 1;
+  s.k_empty = s.k_full + MAX_STAGES;
+  s.s_full = s.k_empty + MAX_STAGES;
+  s.s_free = s.s_full + 4;
+  s.drain = s.s_free + 4;
+  s.tmem_holder = reinterpret_cast<uint32_t *>(s.drain + 1);
+  s.abort_flag = reinterpret_cast<volatile int *>(s.tmem_holder + 1);
+  s.ranges = reinterpret_cast<int *>(s.tmem_holder + 2);
+  return s;
+}
+constexpr size_t BAR_BYTES = (1 + 2 * MAX_STAGES + 4 + 4 + 1) * 8 + 8 + (2 * MAX_RT + 1) * 4;
+
+__device__ __forceinline__ void init_barriers(const Smem &s, const Geo &p) {
+  mbar_init(s.q_full, 1);
+  for (int st = 0; st < p.stages; ++st) {
+    mbar_init(&s.k_full[st], 1);
+    mbar_init(&s.k_empty[st], 1);
+  }
+  for (int b = 0; b < 4; ++b) {
+    mbar_init(&s.s_full[b], 1);
+    mbar_init(&s.s_free[b], 128);
+  }
+  mbar_init(s.drain, 1);
+  *s.abort_flag = 0;
+  fence_mbar_init();
+}
+
+// Key tiles [kt0, kt1) of this CTA's split of the group's visible keys.
+__device__ __forceinline__ void split_range(int kv_end, int split, int splits, int &kt0, int &kt1) {
+  const int n_kt = (kv_end + BKEY - 1) / BKEY;
+  const int per = (n_kt + splits - 1) / splits;
+  kt0 = min(n_kt, split * per);
+  kt1 = min(n_kt, (split + 1) * per);
+}
+
+// warp 0: Q tiles of the group once, then the K tiles [kt0, kt0 + n) through the ring.
+// Pass 1 wants row tile u as one K-major operand (its two 64-wide chunks
+// adjacent); pass 2 wants each 64-wide chunk of all rows as one operand.
+__device__ __forceinline__ void producer(const Smem &s, const Geo &p, const CUtensorMap *tmQ, const CUtensorMap *tmK,
+                                         int g, int kt0, int n, bool chunk_major) {
+  mbar_arrive_expect_tx(s.q_full, p.n_sub * TILE_BYTES);
+  for (int u = 0; u < p.n_sub; ++u) {
+    uint8_t *d0 = chunk_major ? s.q + u * CHUNK_BYTES : s.q + u * TILE_BYTES;
+    uint8_t *d1 = chunk_major ? s.q + (p.n_sub + u) * CHUNK_BYTES : s.q + u * TILE_BYTES + CHUNK_BYTES;
+    tma_load_3d(d0, tmQ, s.q_full, 0, g * p.G, u * p.tq);
+    tma_load_3d(d1, tmQ, s.q_full, 64, g * p.G, u * p.tq);
+  }
+  uint32_t issued = 0, par = 0;
+  for (int i = 0; i < n; ++i) {
+    const int st = i % p.stages;
+    const uint32_t ph = (i / p.stages) & 1;
+    if (!mbar_wait(&s.k_empty[st], ph ^ 1u, s.abort_flag, p.status, p.wait_ns, 0x31u)) break;
+    mbar_arrive_expect_tx(&s.k_full[st], TILE_BYTES);
+    const int key0 = (kt0 + i) * BKEY;
+    tma_load_3d(s.k + st * TILE_BYTES, tmK, &s.k_full[st], 0, g, key0);
+    tma_load_3d(s.k + st * TILE_BYTES + CHUNK_BYTES, tmK, &s.k_full[st], 64, g, key0);
+    issued |= 1u << st;
+    par = (par & ~(1u << st)) | (ph << st);
+  }
+  if (*s.abort_flag) {
+    mbar_drain(s.q_full, 0, p.status);
+    for (int st = 0; st < p.stages; ++st)
+      if (issued & (1u << st)) mbar_drain(&s.k_full[st], (par >> st) & 1u, p.status);
+  }
+}
+
+// warp 1: for each key tile, one 8-MMA group per sub-item into its buffer.
+// Pass 1: D = Q_u K^T (A = row tile u, B = K tile).  Pass 2: D = K Q_u^T
+// (A = K tile, B = column chunk u of the probe rows).
+__device__ __forceinline__ void mma_issuer(const Smem &s, const Geo &p, uint32_t tmem, int n, bool transposed) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+  bool ok = mbar_wait(s.q_full, 0, s.abort_flag, p.status, p.wait_ns, 0x32u);
+  tc_fence_after();
+  const uint32_t q_addr = smem_u32(s.q);
+  for (int i = 0; ok && i < n; ++i) {
+    const int st = i % p.stages;
+    if (!mbar_wait(&s.k_full[st], (i / p.stages) & 1, s.abort_flag, p.status, p.wait_ns, 0x33u)) break;
+    const uint32_t k_addr = smem_u32(s.k + st * TILE_BYTES);
+    for (int u = 0; ok && u < p.n_sub; ++u) {
+      const int b = (i & 1) * 2 + (u & 1);
+      const uint32_t use = buffer_uses(i, u, p.n_sub);
+      if (!mbar_wait(&s.s_free[b], (use & 1u) ^ 1u, s.abort_flag, p.status, p.wait_ns, 0x34u)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t xr[BKEY];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + b * BKEY + c * 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32 * c));
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s_free[b]);
-      const int j0 = (kt0 + i) * BKEY;
-      const bool need_mask = (j0 + BKEY > mask_from) || (j0 + BKEY > kv_end);
-      float x[BKEY], m8[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) m8[t] = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BKEY; ++c) {
-        float v = __uint_as_float(xr[c]) * p.scale_log2;
-        if (need_mask) {
-          const int key = j0 + c;
-          if (!(key < kv_end && __ldg(p.kpos + key) <= qp)) v = -INFINITY;
-        }
-        x[c] = v;
-        m8[c & 7] = fmaxf(m8[c & 7], v);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t kc = k_addr + (kk >> 2) * CHUNK_BYTES;
+        const uint32_t qc = transposed ? q_addr + ((kk >> 2) * p.n_sub + u) * CHUNK_BYTES
+                                       : q_addr + u * TILE_BYTES + (kk >> 2) * CHUNK_BYTES;
+        const uint64_t qd = sdesc_k_sw128(qc) + 2 * (kk & 3), kd = sdesc_k_sw128(kc) + 2 * (kk & 3);
+        mma_bf16_ss(tmem + b * 128, transposed ? kd : qd, transposed ? qd : kd, idesc, kk > 0);
       }
-      const float mt =
-          fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      const float m_new = fmaxf(m, mt);
-      if (m_new == -INFINITY) continue;
-      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < BKEY; ++c) s8[c & 7] += ex2(x[c] - m_new);
-      const float sum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-      l = (m == -INFINITY ? 0.f : l * ex2(m - m_new)) + sum;
-      m = m_new;
+      tc_commit(&s.s_full[b]);
     }
-    if (ok) partial[(static_cast<int64_t>(split) * p.Hkv + g) * p.rows_pad + rt * 128 + r] = make_float2(m, l);
+    if (ok) tc_commit(&s.k_empty[st]);
+  }
+  tc_commit(s.drain);
+  mbar_drain(s.drain, 0, p.status);
+}
+
+// Loads the 128 fp32 columns of buffer b for this warp's 32 lanes, then
+// releases the buffer to the MMA warp.  False when the CTA is aborting.
+__device__ __forceinline__ bool take_buffer(const Smem &s, const Geo &p, uint32_t lane_base, int b, uint32_t use,
+                                            uint32_t (&xr)[128], uint32_t where) {
+  const bool ok = mbar_wait(&s.s_full[b], use & 1u, s.abort_flag, p.status, p.wait_ns, where);
+  if (!__all_sync(0xffffffffu, ok)) return false;
+  tc_fence_after();
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    tmem_ld32(lane_base + b * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32 * c));
+  tmem_ld_wait();
+  tc_fence_before();
+  mbar_arrive(&s.s_free[b]);
+  return true;
+}
+
+__device__ __forceinline__ void search_ranges(const Smem &s, const Geo &p, int n_rt) {
+  // warps 4..11: one search each: row tile u's last probe (kv_end) and
+  // first probe (mask_from)
+  const int w = static_cast<int>(threadIdx.x >> 5) - 4;
+  if (w >= 0 && w < 2 * n_rt) {
+    const int u = w >> 1;
+    const int first = u * p.tq, last = min(first + p.tq, p.P) - 1;
+    const int r = warp_upper_bound(p.kpos, p.Nc, p.ppos[(w & 1) ? first : last]);
+    if ((threadIdx.x & 31) == 0) s.ranges[(w & 1) ? MAX_RT + u : u] = r;
+  }
+}
+
+// ------------------------------------------------------------------ pass 1
+__global__ void __launch_bounds__(THREADS, 1)
+    probe_stats_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ Geo p, float2 *__restrict__ partial) {
+  extern __shared__ uint8_t smem_raw[];
+  const Smem s = carve_smem(smem_raw, p, false);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x % p.splits;
+  const int g = blockIdx.x / p.splits;
+  const int n_rt = p.n_sub;
+
+  if (threadIdx.x == 0) init_barriers(s, p);
+  if (warp == 1) {
+    tmem_alloc(s.tmem_holder, 512);
+    tmem_relinquish();
+  }
+  search_ranges(s, p, n_rt);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s.tmem_holder;
+  const int kv_group = s.ranges[n_rt - 1];  // the last row tile sees the most keys
+  int kt0, kt1;
+  split_range(kv_group, split, p.splits, kt0, kt1);
+  const int n = kt1 - kt0;
+
+  if (warp == 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
+    if (lane == 0) producer(s, p, &tmQ, &tmK, g, kt0, n, false);
+    __syncwarp();
+  } else if (warp == 1) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
+    if (lane == 0) mma_issuer(s, p, tmem, n, false);
+    __syncwarp();
+  } else if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));  // idle
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_HIGH));
+    const int wg = (warp - 4) >> 2;
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float c2 = p.scale_log2;
+    float m[MAX_RT], l[MAX_RT];
+#pragma unroll
+    for (int q = 0; q < MAX_RT; ++q) {
+      m[q] = -INFINITY;
+      l[q] = 0.f;
+    }
+    bool ok = true;
+    for (int i = wg; ok && i < n; i += 2) {
+      const int j0 = (kt0 + i) * BKEY;
+      for (int u = 0; u < n_rt; ++u) {
+        const int b = wg * 2 + (u & 1);
+        uint32_t xr[128];
+        if (!take_buffer(s, p, lane_base, b, buffer_uses(i, u, n_rt), xr, 0x35u)) {
+          ok = false;
+          break;
+        }
+        const int kv_end = s.ranges[u], mask_from = s.ranges[MAX_RT + u];
+        if (j0 + BKEY > mask_from || j0 + BKEY > kv_end) {
+          const int pr = u * p.tq + r / p.G;
+          const int32_t qp = pr < p.P ? p.ppos[pr] : INT_MIN;
+#pragma unroll
+          for (int c = 0; c < BKEY; ++c) {
+            const int key = j0 + c;
+            if (!(key < kv_end && __ldg(p.kpos + key) <= qp)) xr[c] = 0xff800000u;  // -inf
+          }
+        }
+        float m8[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) m8[t] = __uint_as_float(xr[t]);
+#pragma unroll
+        for (int c = 8; c < BKEY; c += 2)
+          m8[(c >> 1) & 7] = fmax3(m8[(c >> 1) & 7], __uint_as_float(xr[c]), __uint_as_float(xr[c + 1]));
+        const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * c2;
+        float mu = m[0], lu = l[0];
+#pragma unroll
+        for (int q = 1; q < MAX_RT; ++q)
+          if (q == u) {
+            mu = m[q];
+            lu = l[q];
+          }
+        const float m_new = fmaxf(mu, mt);
+        if (m_new == -INFINITY) continue;  // nothing visible yet
+        const float neg = -m_new;
+        float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < BKEY; ++c) s8[c & 7] += ex2(fmaf(__uint_as_float(xr[c]), c2, neg));
+        const float sum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+        lu = (mu == -INFINITY ? 0.f : lu * ex2(mu - m_new)) + sum;
+#pragma unroll
+        for (int q = 0; q < MAX_RT; ++q)
+          if (q == u) {
+            m[q] = m_new;
+            l[q] = lu;
+          }
+      }
+    }
+    if (ok) {
+#pragma unroll
+      for (int q = 0; q < MAX_RT; ++q)
+        if (q < n_rt)
+          partial[(static_cast<int64_t>(split * 2 + wg) * p.Hkv + g) * p.rows_pad + q * 128 + r] =
+              make_float2(m[q], l[q]);
+    }
   }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
-// merge the splits: stats[g][row].x = max + log2(sum) in log2 units
-__global__ void probe_combine_kernel(const float2 *__restrict__ partial, int splits, int total,
+// merge the partials: stats[g][row].x = max + log2(sum) in log2 units
+__global__ void probe_combine_kernel(const float2 *__restrict__ partial, int parts, int total,
                                      float2 *__restrict__ stats) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= total) return;
   float m = -INFINITY;
-  for (int s = 0; s < splits; ++s) m = fmaxf(m, partial[static_cast<int64_t>(s) * total + i].x);
+  for (int s = 0; s < parts; ++s) m = fmaxf(m, partial[static_cast<int64_t>(s) * total + i].x);
   float l = 0.f;
   if (m != -INFINITY)
-    for (int s = 0; s < splits; ++s) {
+    for (int s = 0; s < parts; ++s) {
       const float2 v = partial[static_cast<int64_t>(s) * total + i];
       if (v.x != -INFINITY) l += v.y * ex2(v.x - m);
     }
@@ -240,194 +381,122 @@ __global__ void probe_combine_kernel(const float2 *__restrict__ partial, int spl
 }
 
 // ------------------------------------------------------------------ pass 2
-constexpr int P2_STAGES = 2;
-constexpr int P2_MAX_ROWS = 512;
-
 __global__ void __launch_bounds__(THREADS, 1)
     probe_scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ Geo p, int chunks, const float2 *__restrict__ stats,
-                        float *__restrict__ group) {
+                        const __grid_constant__ Geo p, const float2 *__restrict__ stats, float *__restrict__ group) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int ncol = p.rows_pad;                 // probe rows of this group (padded), <= 512
-  const int q_tiles = ncol / 128;
-  uint8_t *sQ = smem;                          // q_tiles x 32 KB: rows [ncol] as 64-wide chunks per tile
-  uint8_t *sK = smem + q_tiles * TILE_BYTES;   // P2_STAGES x 32 KB
-  float *smm = reinterpret_cast<float *>(sK + P2_STAGES * TILE_BYTES);   // per column: max + log2(sum)
-  int32_t *scol = reinterpret_cast<int32_t *>(smm + P2_MAX_ROWS);      // per column: probe position
-  uint64_t *bars = reinterpret_cast<uint64_t *>(scol + P2_MAX_ROWS);
-  uint64_t *q_full = bars, *k_full = bars + 1, *k_empty = bars + 1 + P2_STAGES, *s_full = bars + 1 + 2 * P2_STAGES,
-           *s_free = s_full + 2, *drain = s_free + 2;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-  int *s_range = reinterpret_cast<int *>(tmem_holder + 2);
-
+  const Smem s = carve_smem(smem_raw, p, true);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x % chunks;
-  const int g = blockIdx.x / chunks;
-  // the probe rows are processed in chunks of CW columns, one TMEM buffer each
-  const int CW = (ncol % 256 == 0) ? 256 : 128;
-  const int nch = ncol / CW;
-  const uint32_t tmem_cols = 512;
+  const int split = blockIdx.x % p.splits;
+  const int g = blockIdx.x / p.splits;
+  const int ncol = p.rows_pad;
 
-  for (int c = threadIdx.x; c < P2_MAX_ROWS; c += THREADS) {
+  for (int c = threadIdx.x; c < MAX_RT * 128; c += THREADS) {
     const int pr = c / p.G;
     const bool live = c < ncol && pr < p.P;
-    smm[c] = live ? stats[g * ncol + c].x : INFINITY;
-    scol[c] = live ? p.ppos[pr] : INT_MIN;
+    s.colv[c] = live ? stats[g * ncol + c].x : INFINITY;
+    s.colp[c] = live ? p.ppos[pr] : INT_MIN;
   }
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < P2_STAGES; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 128);
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-    const int kv_end = upper_bound(p.kpos, p.Nc, p.ppos[p.P - 1]);
-    const int n_kt = (kv_end + BKEY - 1) / BKEY;
-    const int per = (n_kt + chunks - 1) / chunks;
-    s_range[0] = min(n_kt, chunk * per);
-    s_range[1] = min(n_kt, (chunk + 1) * per);
-    s_range[2] = kv_end;
-  }
+  if (threadIdx.x == 0) init_barriers(s, p);
   if (warp == 1) {
-    tmem_alloc(tmem_holder, tmem_cols);
+    tmem_alloc(s.tmem_holder, 512);
     tmem_relinquish();
+  }
+  if (warp == 4) {
+    const int r = warp_upper_bound(p.kpos, p.Nc, p.ppos[p.P - 1]);
+    if (lane == 0) s.ranges[2 * MAX_RT] = r;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  const int kt0 = s_range[0], kt1 = s_range[1], kv_end = s_range[2];
+  const uint32_t tmem = *s.tmem_holder;
+  const int kv_end = s.ranges[2 * MAX_RT];
+  int kt0, kt1;
+  split_range(kv_end, split, p.splits, kt0, kt1);
   const int n = kt1 - kt0;
   const int32_t ppos_min = p.ppos[0];
 
   if (warp == 0) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, q_tiles * TILE_BYTES);
-      for (int t = 0; t < q_tiles; ++t) {
-        // chunk c of every probe row lives at sQ + c*(q_tiles*16KB) + t*16KB, so each
-        // 64-wide chunk is one K-major operand of ncol rows
-        tma_load_3d(sQ + t * CHUNK_BYTES, &tmQ, q_full, 0, g * p.G, t * p.tq);
-        tma_load_3d(sQ + q_tiles * CHUNK_BYTES + t * CHUNK_BYTES, &tmQ, q_full, 64, g * p.G, t * p.tq);
-      }
-      uint32_t issued = 0, par = 0;
-      for (int i = 0; i < n; ++i) {
-        const int st = i % P2_STAGES;
-        const uint32_t ph = (i / P2_STAGES) & 1;
-        if (!mbar_wait(&k_empty[st], ph ^ 1u, abort_flag, p.status, p.wait_ns, 0x41u)) break;
-        mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
-        const int key0 = (kt0 + i) * BKEY;
-        tma_load_3d(sK + st * TILE_BYTES, &tmK, &k_full[st], 0, g, key0);
-        tma_load_3d(sK + st * TILE_BYTES + CHUNK_BYTES, &tmK, &k_full[st], 64, g, key0);
-        issued |= 1u << st;
-        par = (par & ~(1u << st)) | (ph << st);
-      }
-      if (*abort_flag) {
-        mbar_drain(q_full, 0, p.status);
-        for (int st = 0; st < P2_STAGES; ++st)
-          if (issued & (1u << st)) mbar_drain(&k_full[st], (par >> st) & 1u, p.status);
-      }
-    }
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
+    if (lane == 0) producer(s, p, &tmQ, &tmK, g, kt0, n, true);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, CW, 0, 0);
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status, p.wait_ns, 0x42u);
-      tc_fence_after();
-      // work item it = (key tile it / nch, column chunk it % nch) into TMEM buffer it % 2
-      for (int it = 0; ok && it < n * nch; ++it) {
-        const int i = it / nch, h = it % nch;
-        const int st = i % P2_STAGES;
-        const int b = it & 1;
-        if (!mbar_wait(&s_free[b], ((it >> 1) & 1) ^ 1u, abort_flag, p.status, p.wait_ns, 0x43u)) break;
-        if (h == 0 && !mbar_wait(&k_full[st], (i / P2_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x44u)) break;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + st * TILE_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sdesc_k_sw128(k_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3);
-          const uint32_t q_addr = smem_u32(sQ + (kk >> 2) * q_tiles * CHUNK_BYTES + h * (CW / 128) * CHUNK_BYTES);
-          mma_bf16_ss(tmem + b * CW, a, sdesc_k_sw128(q_addr) + 2 * (kk & 3), idesc, kk > 0);
-        }
-        if (h == nch - 1) tc_commit(&k_empty[st]);
-        tc_commit(&s_full[b]);
-      }
-      tc_commit(drain);
-      mbar_drain(drain, 0, p.status);
-    }
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
+    if (lane == 0) mma_issuer(s, p, tmem, n, true);
     __syncwarp();
+  } else if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));  // idle
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_HIGH));
+    const int wg = (warp - 4) >> 2;
     const int quad = warp & 3;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float c2 = p.scale_log2;
     bool ok = true;
-    float acc = 0.f;
-    for (int it = 0; it < n * nch; ++it) {
-      const int i = it / nch, h = it % nch;
-      const int b = it & 1;
-      ok = mbar_wait(&s_full[b], (it >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x45u);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+    for (int i = wg; ok && i < n; i += 2) {
       const int j = (kt0 + i) * BKEY + quad * 32 + lane;
       const bool live = j < kv_end;
       const int32_t kp = live ? __ldg(p.kpos + j) : INT_MAX;
       const bool all_vis = kp <= ppos_min;
-      if (h == 0) acc = 0.f;
       float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-      for (int c0 = 0; c0 < CW; c0 += 32) {
-        uint32_t xr[32];
-        tmem_ld32(lane_base + b * CW + c0, xr);
-        tmem_ld_wait();
-        const float *mmc = smm + h * CW + c0;
+      for (int u = 0; u < p.n_sub; ++u) {
+        const int b = wg * 2 + (u & 1);
+        uint32_t xr[128];
+        if (!take_buffer(s, p, lane_base, b, buffer_uses(i, u, p.n_sub), xr, 0x45u)) {
+          ok = false;
+          break;
+        }
+        const float *cv = s.colv + u * 128;
+        if (all_vis) {
 #pragma unroll
-        for (int t = 0; t < 32; t += 4) {
-          const float4 mq = *reinterpret_cast<const float4 *>(mmc + t);
-          const float mv[4] = {mq.x, mq.y, mq.z, mq.w};
+          for (int t = 0; t < 128; t += 4) {
+            const float4 mq = *reinterpret_cast<const float4 *>(cv + t);
+            a4[0] += ex2(fmaf(__uint_as_float(xr[t + 0]), c2, -mq.x));
+            a4[1] += ex2(fmaf(__uint_as_float(xr[t + 1]), c2, -mq.y));
+            a4[2] += ex2(fmaf(__uint_as_float(xr[t + 2]), c2, -mq.z));
+            a4[3] += ex2(fmaf(__uint_as_float(xr[t + 3]), c2, -mq.w));
+          }
+        } else {
+          const int32_t *cp = s.colp + u * 128;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float w = ex2(fmaf(__uint_as_float(xr[t + e]), p.scale_log2, -mv[e]));
-            if (!all_vis && kp > scol[h * CW + c0 + t + e]) w = 0.f;
-            a4[e] += w;
+          for (int t = 0; t < 128; ++t) {
+            const float w = ex2(fmaf(__uint_as_float(xr[t]), c2, -cv[t]));
+            a4[t & 3] += kp > cp[t] ? 0.f : w;
           }
         }
       }
-      acc += (a4[0] + a4[1]) + (a4[2] + a4[3]);
-      tc_fence_before();
-      mbar_arrive(&s_free[b]);
-      if (h == nch - 1 && live) group[static_cast<int64_t>(g) * p.Nc + j] = acc;
+      if (ok && live) group[static_cast<int64_t>(g) * p.Nc + j] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
     }
     // keys beyond every probe position get no weight
-    if (ok) {
-      const int first = kv_end;
-      for (int jj = first + (threadIdx.x - 64); jj < p.Nc && chunk == chunks - 1; jj += 128)
+    if (ok && split == p.splits - 1)
+      for (int jj = kv_end + (static_cast<int>(threadIdx.x) - 128); jj < p.Nc; jj += THREADS - 128)
         group[static_cast<int64_t>(g) * p.Nc + jj] = 0.f;
-    }
   }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, tmem_cols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
 int rows_pad_of(int P, int G) { return ((P * G + 127) / 128) * 128; }
 
+size_t smem_bytes(int n_sub, int stages, bool cols) {
+  return 1024 + static_cast<size_t>(n_sub + stages) * TILE_BYTES + (cols ? MAX_RT * 128 * 8 : 0) + BAR_BYTES;
+}
+int stages_for(int n_sub, bool cols) {
+  int st = MAX_STAGES;
+  while (st > 2 && smem_bytes(n_sub, st, cols) > static_cast<size_t>(SMEM_CAP)) --st;
+  return st;
+}
+
 }  // namespace
 
 size_t probe_bf16_stats_bytes(int P, int Hq, int64_t) {
+  // partials of both warpgroups of every split plus the combined statistics;
   // worst case over G: Hkv * rows_pad <= Hq * P + 127 * Hq
   const size_t rows = static_cast<size_t>(Hq) * P + 127 * static_cast<size_t>(Hq);
-  return (MAX_SPLITS + 1) * rows * sizeof(float2);
+  return (2 * MAX_SPLITS + 1) * rows * sizeof(float2);
 }
 
 spts_status launch_probe_bf16(const void *q, const int32_t *qpos, int P, const void *k, const int32_t *kpos,
@@ -436,7 +505,7 @@ spts_status launch_probe_bf16(const void *q, const int32_t *qpos, int P, const v
   const int G = Hq / Hkv;
   const int tq = 128 / G;
   const int rows_pad = rows_pad_of(P, G);
-  if (rows_pad > P2_MAX_ROWS) {
+  if (rows_pad > MAX_RT * 128) {
     set_error("spts_probe_scores: P * (Hq/Hkv) must be <= 512 on the bf16 path (got %d)", P * G);
     return SPTS_ERR_UNSUPPORTED;
   }
@@ -455,6 +524,7 @@ spts_status launch_probe_bf16(const void *q, const int32_t *qpos, int P, const v
     SPTS_TRY(make_tmap(&tk_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, strides, box,
                        CU_TENSOR_MAP_SWIZZLE_128B));
   }
+  const int n_kt = static_cast<int>((Nc + BKEY - 1) / BKEY);
   Geo geo{};
   geo.ppos = qpos;
   geo.kpos = kpos;
@@ -465,34 +535,35 @@ spts_status launch_probe_bf16(const void *q, const int32_t *qpos, int P, const v
   geo.G = G;
   geo.tq = tq;
   geo.rows_pad = rows_pad;
+  geo.n_sub = rows_pad / 128;
+  geo.splits = std::max(1, std::min(std::min(num_sms() / Hkv, MAX_SPLITS), n_kt));
   geo.scale_log2 = scale * LOG2E;
   geo.status = status;
   geo.wait_ns = wait_limit_ns();
 
-  const int n_rt = rows_pad / 128;
-  const int n_kt = static_cast<int>((Nc + BKEY - 1) / BKEY);
-  int splits = (2 * num_sms() + n_rt * Hkv - 1) / (n_rt * Hkv);
-  splits = std::max(1, std::min(std::min(splits, MAX_SPLITS), n_kt));
+  const int parts = 2 * geo.splits;
   float2 *partial = reinterpret_cast<float2 *>(row_stats);
-  float2 *stats = partial + static_cast<size_t>(splits) * Hkv * rows_pad;
+  float2 *stats = partial + static_cast<size_t>(parts) * Hkv * rows_pad;
 
+  Geo g1 = geo;
+  g1.stages = stages_for(geo.n_sub, false);
+  const size_t sm1 = smem_bytes(geo.n_sub, g1.stages, false);
   SPTS_CUDA_TRY(cudaFuncSetAttribute(probe_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(P1_SMEM)));
-  probe_stats_kernel<<<n_rt * Hkv * splits, THREADS, P1_SMEM, s>>>(tq_map, tk_map, geo, n_rt, splits, partial);
+                                     static_cast<int>(sm1)));
+  probe_stats_kernel<<<Hkv * geo.splits, THREADS, sm1, s>>>(tq_map, tk_map, g1, partial);
   note_launch();
   SPTS_CUDA_TRY(cudaGetLastError());
   const int total = Hkv * rows_pad;
-  probe_combine_kernel<<<(total + 255) / 256, 256, 0, s>>>(partial, splits, total, stats);
+  probe_combine_kernel<<<(total + 255) / 256, 256, 0, s>>>(partial, parts, total, stats);
   note_launch();
   SPTS_CUDA_TRY(cudaGetLastError());
 
-  const size_t p2_smem = 1024 + static_cast<size_t>(rows_pad / 128) * TILE_BYTES + P2_STAGES * TILE_BYTES +
-                         P2_MAX_ROWS * (sizeof(float2) + sizeof(int32_t)) + 256;
-  int chunks = (2 * num_sms() + Hkv - 1) / Hkv;
-  chunks = std::max(1, std::min(chunks, n_kt));
+  Geo g2 = geo;
+  g2.stages = stages_for(geo.n_sub, true);
+  const size_t sm2 = smem_bytes(geo.n_sub, g2.stages, true);
   SPTS_CUDA_TRY(cudaFuncSetAttribute(probe_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(p2_smem)));
-  probe_scores_kernel<<<Hkv * chunks, THREADS, p2_smem, s>>>(tq_map, tk_map, geo, chunks, stats, group);
+                                     static_cast<int>(sm2)));
+  probe_scores_kernel<<<Hkv * geo.splits, THREADS, sm2, s>>>(tq_map, tk_map, g2, stats, group);
   note_launch();
   SPTS_CUDA_TRY(cudaGetLastError());
   return SPTS_OK;
