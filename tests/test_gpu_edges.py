@@ -24,6 +24,18 @@ def test_select_all_equal_scores_takes_lowest_indices():
     assert np.array_equal(idx.cpu().numpy(), want)
 
 
+
+@pytest.mark.parametrize("Nc,k,tail", [(100000, 20000, 128), (70000, 70000, 64), (70000, 64, 64), (50000, 1, 0)])
+def test_select_large_sets_on_the_grid_path(Nc, k, tail):
+    # above 48K free candidates the selection runs on the grid; all-equal
+    # scores put every key in one radix bin, few distinct values make long
+    # runs of ties at the threshold
+    for s in (np.full(Nc, 0.125, np.float32), rng.integers(0, 5, Nc).astype(np.float32) * 0.5):
+        want, _ = O.select_topk(s, k, tail)
+        idx = S.spts_select_topk(torch.from_numpy(s).cuda(), k, tail)
+        assert np.array_equal(idx.cpu().numpy(), want)
+
+
 def test_select_zero_scores_and_negative_zero():
     s = torch.zeros(300, device="cuda")
     s[::3] = -0.0

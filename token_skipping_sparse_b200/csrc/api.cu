@@ -95,7 +95,9 @@ spts_status spts_ltp_scores(spts_dtype dt, const void *x, int64_t Nc, int D, con
 }
 
 // ------------------------------------------------------------------ select
-size_t spts_select_topk_workspace(int64_t) { return kStatusBytes; }
+size_t spts_select_topk_workspace(int64_t Nc) {
+  return kStatusBytes + Carver::round(topk_scratch_bytes(Nc));
+}
 
 spts_status spts_select_topk(const float *s_a, const float *s_b, spts_fuse mode, float w_a, float w_b,
                              int64_t Nc, int64_t k, int64_t force_tail, int32_t *idx_out, float *fused_out,
@@ -112,8 +114,10 @@ spts_status spts_select_topk(const float *s_a, const float *s_b, spts_fuse mode,
                "%s: misaligned pointer", who);
   SPTS_TRY(check_ws(ws, ws_bytes, spts_select_topk_workspace(Nc), who));
   if (Nc == 0) return SPTS_OK;
+  Carver cv(ws, ws_bytes);
+  void *scratch = cv.take(topk_scratch_bytes(Nc));
   return launch_select_topk(s_a, s_b, mode, w_a, w_b, Nc, k, force_tail, idx_out, fused_out, kth_score_out,
-                            static_cast<uint32_t *>(ws), cs(stream));
+                            cv.status(), scratch, cs(stream));
 }
 
 // ------------------------------------------------------------------ attention
@@ -177,7 +181,9 @@ spts_status spts_reduced_ffn(spts_dtype dt, float *h, int64_t Nc, int D, const i
 }
 
 // ------------------------------------------------------------------ MSDP prune
-size_t spts_stage_prune_workspace(int64_t Nc) { return kStatusBytes + Carver::round(Nc * sizeof(int32_t)); }
+size_t spts_stage_prune_workspace(int64_t Nc) {
+  return kStatusBytes + Carver::round(Nc * sizeof(int32_t)) + Carver::round(topk_scratch_bytes(Nc));
+}
 
 spts_status spts_stage_prune(const float *scores, int64_t Nc, int64_t k_keep, int64_t force_tail,
                              const float *h_in, const int32_t *pos_in, int D, float *h_out, int32_t *pos_out,
@@ -198,9 +204,10 @@ spts_status spts_stage_prune(const float *scores, int64_t Nc, int64_t k_keep, in
   Carver cv(ws, ws_bytes);
   int32_t *kept = static_cast<int32_t *>(cv.take(Nc * sizeof(int32_t)));
   if (kept_idx) kept = kept_idx;
+  void *scratch = cv.take(topk_scratch_bytes(Nc));
   cudaStream_t s = cs(stream);
   SPTS_TRY(launch_select_topk(scores, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, Nc, k_keep, force_tail, kept, nullptr,
-                              nullptr, cv.status(), s));
+                              nullptr, cv.status(), scratch, s));
   return launch_gather_rows(h_in, Nc, kept, k_keep, static_cast<int64_t>(D) * 4, h_out, pos_in, pos_out,
                             cv.status(), s);
 }

@@ -15,6 +15,7 @@ struct LayerBufs {
   void *xn, *kk, *vv, *qprobe, *xsel, *qsel, *osel, *act;
   float *s, *group, *stats, *c, *f;
   int32_t *idx_a, *idx_f, *qpos;
+  void *topk;  // scratch of the grid top-k
 };
 
 // Carves the workspace; with cv.base == nullptr it only measures.
@@ -37,6 +38,7 @@ void carve(Carver &cv, const spts_layer_desc *L, int64_t Nc, LayerBufs &b) {
   b.idx_a = static_cast<int32_t *>(cv.take(k * 4));
   b.idx_f = static_cast<int32_t *>(cv.take(k * 4));
   b.qpos = static_cast<int32_t *>(cv.take(k * 4));
+  b.topk = cv.take(topk_scratch_bytes(Nc));
 }
 
 // A side stream and fork/join events per (host thread, device): the V and
@@ -173,7 +175,8 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
                              s));
   SPTS_TRY(launch_sum_groups(b.group, L->Hkv, Nc, sc, s));
   SPTS_TRY(mark(5));
-  SPTS_TRY(launch_select_topk(sc, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, Nc, k, P, idx_a, nullptr, nullptr, st, s));
+  SPTS_TRY(launch_select_topk(sc, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, Nc, k, P, idx_a, nullptr, nullptr, st, b.topk,
+                              s));
   SPTS_TRY(mark(6));
 
   // a5-a7: Q for the selected rows, reduced attention, O projection into h
@@ -206,7 +209,7 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   SPTS_TRY(mark(11));
   SPTS_TRY(launch_ltp_bf16(b.xn, Nc, D, W->ltp_a, L->r, W->ltp_b, D, c, st, s));
   SPTS_TRY(mark(12));
-  SPTS_TRY(launch_select_topk(sc, c, L->fuse, L->w_a, L->w_b, Nc, k, P, idx_f, f, nullptr, st, s));
+  SPTS_TRY(launch_select_topk(sc, c, L->fuse, L->w_a, L->w_b, Nc, k, P, idx_f, f, nullptr, st, b.topk, s));
   SPTS_TRY(launch_gather_rows(b.xn, Nc, idx_f, k, static_cast<int64_t>(D) * 2, b.xsel, nullptr, nullptr, st, s));
   SPTS_TRY(mark(13));
   GemmArgs g1{b.xsel, k, D, W->w_gate, W->w_up, L->F, SPTS_EPI_SWIGLU, b.act, nullptr, nullptr, 0.0, st};
@@ -270,7 +273,12 @@ spts_status spts_msdp_forward(const spts_layer_desc *L, const spts_layer_weights
     o.f = f;
     for (int l = 0; l < layers_per_stage; ++l, ++li) SPTS_TRY(spts_layer_forward(&d, &W[li], ha, pa, Nc, &o, ws, lw, stream));
     // stage boundary: C_{s+1} = top-k_s of C_s by the last layer's fused score
-    SPTS_TRY(launch_select_topk(f, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, Nc, d.k, L->P, kept, nullptr, nullptr, st, s));
+    // the layers are done with their workspace: its top-k scratch serves the prune
+    Carver lcv(ws, lw);
+    LayerBufs lb;
+    carve(lcv, &lmax, N, lb);
+    SPTS_TRY(launch_select_topk(f, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, Nc, d.k, L->P, kept, nullptr, nullptr, st,
+                                lb.topk, s));
     SPTS_TRY(launch_gather_rows(ha, Nc, kept, d.k, static_cast<int64_t>(L->D) * 4, hb, pa, pb, st, s));
     if (stage_pos)
       SPTS_CUDA_TRY(cudaMemcpyAsync(stage_pos + out_off, pb, static_cast<size_t>(d.k) * 4, cudaMemcpyDeviceToDevice, s));

@@ -72,6 +72,6 @@ extern "C" spts_status spts_stage_prune_noalloc(const float *scores, int64_t Nc,
   // nothing in the scratch has to start at zero.  No status word is kept:
   // device-side index checks report nothing in this variant.
   SPTS_TRY(launch_select_topk(scores, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, Nc, k_keep, force_tail, kept, nullptr,
-                              nullptr, nullptr, s));
+                              nullptr, nullptr, nullptr, s));  // no scratch: the single-CTA selection
   return launch_gather_rows(h_in, Nc, kept, k_keep, static_cast<int64_t>(D) * 4, h_out, pos_in, pos_out, nullptr, s);
 }

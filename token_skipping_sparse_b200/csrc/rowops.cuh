@@ -28,10 +28,13 @@ spts_status launch_inject_salience(void *k, int64_t Nc, const void *q_probe, int
 spts_status launch_gather_i32(const int32_t *src, const int32_t *idx, int64_t m, int32_t *dst, cudaStream_t s);
 spts_status launch_sum_groups(const float *group, int G, int64_t n, float *s, cudaStream_t st);
 
-// Top-k selection (single CTA radix select + stable compaction).
+// Top-k selection: radix select + stable compaction, on one CTA, or on the
+// grid when `scratch` (topk_scratch_bytes(Nc) bytes) is given and the
+// candidate set is large.
+size_t topk_scratch_bytes(int64_t Nc);
 spts_status launch_select_topk(const float *s_a, const float *s_b, int mode, float w_a, float w_b, int64_t Nc,
                                int64_t k, int64_t force_tail, int32_t *idx_out, float *fused_out,
-                               float *kth_out, uint32_t *status, cudaStream_t s);
+                               float *kth_out, uint32_t *status, void *scratch, cudaStream_t s);
 
 // fp32 CUDA-core attention paths.
 spts_status launch_probe_f32(const float *q, const int32_t *qpos, int P, const float *k, const int32_t *kpos,

@@ -23,6 +23,9 @@ namespace spts {
 constexpr int TK_THREADS = 1024;
 constexpr int TK_ITEMS = 8;
 constexpr int TK_SMEM_KEYS = 49152;  // 192 KB of cached keys
+#ifndef TK_GRID_MIN
+#define TK_GRID_MIN 49152  // above this many free candidates the grid path runs (given scratch)
+#endif
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
@@ -224,11 +227,340 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
   if (tid == 0 && kth_out) *kth_out = k_free > 0 ? key_value(T) : __uint_as_float(0x7FC00000u);
 }
 
+
+// ------------------------------------------------------------------ grid path
+// For large candidate sets the single CTA above streams every pass from L2
+// through one SM.  The grid path spreads the work:
+//   topk_prep_kernel      (grid)   zeroes the top-digit histogram; block
+//                                  maxima of both scores (MAXNORM_ADD);
+//   topk_keys_kernel      (grid)   maxima of the block maxima, fused score,
+//                                  key per candidate into the scratch buffer,
+//                                  histogram of the top 11 key bits;
+//   topk_threshold_kernel (1 CTA)  the bin of the (k - tail)-th largest key,
+//                                  then two more radix digits (11 + 10 bits)
+//                                  over the keys: the threshold T and how
+//                                  many keys equal to T are taken;
+//   topk_count_kernel     (grid)   per chunk, the keys > T and == T;
+//   topk_write_kernel     (grid)   the counts of the chunks before its own,
+//                                  then stable compaction of its chunk; CTA 0
+//                                  appends the forced tail.
+// The result is identical to the single-CTA path (same keys, same threshold,
+// same index order).
+constexpr int TG_THREADS = 1024;
+constexpr int TG_MAX_CTAS = 256;
+constexpr int TG_BINS = 2048;
+constexpr int TG_LOADS = 8;
+
+struct TopkScratch {
+  uint32_t *keys;     // [n_free]
+  uint32_t *hist;     // [TG_BINS]
+  float *maxpart;     // [2][TG_MAX_CTAS]
+  uint32_t *chunk;    // [2][TG_MAX_CTAS]: per chunk, keys > T and keys == T
+  uint32_t *sel;      // [4]: T, need_eq
+};
+
+__host__ __device__ inline size_t tg_round(size_t b) { return (b + 255) & ~size_t(255); }
+
+__host__ __device__ inline TopkScratch tg_carve(void *base, int64_t n_free) {
+  uint8_t *p = static_cast<uint8_t *>(base);
+  TopkScratch t;
+  t.keys = reinterpret_cast<uint32_t *>(p);
+  p += tg_round(static_cast<size_t>(n_free) * 4);
+  t.hist = reinterpret_cast<uint32_t *>(p);
+  p += tg_round(TG_BINS * 4);
+  t.maxpart = reinterpret_cast<float *>(p);
+  p += tg_round(2 * TG_MAX_CTAS * 4);
+  t.chunk = reinterpret_cast<uint32_t *>(p);
+  p += tg_round(4 * TG_MAX_CTAS * 4);
+  t.sel = reinterpret_cast<uint32_t *>(p);
+  return t;
+}
+
+__global__ void __launch_bounds__(TG_THREADS)
+    topk_prep_kernel(FuseArgs fa, int64_t Nc, int64_t chunk, TopkScratch t) {
+  __shared__ float red[2][32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int b = blockIdx.x * TG_THREADS + tid; b < TG_BINS; b += gridDim.x * TG_THREADS) t.hist[b] = 0u;
+  if (fa.mode != SPTS_FUSE_MAXNORM_ADD) return;
+  const int64_t i0 = blockIdx.x * chunk, i1 = min(Nc, i0 + chunk);
+  float ma = -INFINITY, mb = -INFINITY;
+  for (int64_t i = i0 + tid; i < i1; i += TG_THREADS) {
+    ma = fmaxf(ma, __ldg(fa.sa + i));
+    mb = fmaxf(mb, __ldg(fa.sb + i));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, o));
+    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+  }
+  if (lane == 0) {
+    red[0][w] = ma;
+    red[1][w] = mb;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int k = 1; k < 32; ++k) {
+      ma = fmaxf(ma, red[0][k]);
+      mb = fmaxf(mb, red[1][k]);
+    }
+    t.maxpart[blockIdx.x] = ma;
+    t.maxpart[TG_MAX_CTAS + blockIdx.x] = mb;
+  }
+}
+
+
+// Adds 1 to h[bin] for every lane of the warp, one shared-memory atomic per
+// distinct bin (the scores of a layer crowd into few top-digit bins).
+__device__ __forceinline__ void warp_hist_add(uint32_t *h, uint32_t bin, bool active) {
+  const uint32_t act = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const uint32_t peers = __match_any_sync(act, bin);
+  if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+}
+
+__global__ void __launch_bounds__(TG_THREADS)
+    topk_keys_kernel(FuseArgs fa, int64_t Nc, int64_t n_free, int64_t chunk, int n_cta, TopkScratch t,
+                     float *__restrict__ fused_out, uint32_t *status) {
+  __shared__ uint32_t h[TG_BINS];
+  __shared__ float mx[2];
+  const int tid = threadIdx.x;
+  if (fa.mode == SPTS_FUSE_MAXNORM_ADD) {
+    if (tid < 64) {
+      const int which = tid >> 5, lane = tid & 31;
+      float m = -INFINITY;
+      for (int c = lane; c < n_cta; c += 32) m = fmaxf(m, t.maxpart[which * TG_MAX_CTAS + c]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) mx[which] = m;
+    }
+  }
+  for (int b = tid; b < TG_BINS; b += TG_THREADS) h[b] = 0u;
+  __syncthreads();
+  if (fa.mode == SPTS_FUSE_MAXNORM_ADD) {
+    fa.ma = mx[0];
+    fa.mb = mx[1];
+  }
+  const int64_t i0 = blockIdx.x * chunk, i1 = min(Nc, i0 + chunk);
+  for (int64_t base = i0; base < i1; base += TG_THREADS) {
+    const int64_t i = base + tid;
+    uint32_t key = 0u;
+    bool counted = false;
+    if (i < i1) {
+      const float f = fused(fa, i);
+      if (!isfinite(f)) raise_status(status, SPTS_DEV_BADINDEX, 0x71u, static_cast<uint32_t>(i));
+      if (fused_out) fused_out[i] = f;
+      if (i < n_free) {
+        key = order_key(f);
+        t.keys[i] = key;
+        counted = true;
+      }
+    }
+    warp_hist_add(h, key >> 21, counted);
+  }
+  __syncthreads();
+  for (int b = tid; b < TG_BINS; b += TG_THREADS)
+    if (h[b]) atomicAdd(&t.hist[b], h[b]);
+}
+
+// With the bins in descending order, finds the bin holding the krem-th
+// largest of the counted keys; *digit = that bin, *krem_out = its rank
+// inside the bin.  nb = 1024 or 2048 bins, 1024 threads.
+__device__ __forceinline__ void tg_find_bin(const uint32_t *h, int nb, uint32_t krem, uint32_t *warp_tot,
+                                            uint32_t *total, uint32_t *digit, uint32_t *krem_out) {
+  const int tid = threadIdx.x;
+  const int per = nb / TG_THREADS;  // 1 or 2 bins per thread, highest bins first
+  uint32_t c0 = h[nb - 1 - tid * per], c1 = per == 2 ? h[nb - 2 - tid * per] : 0u;
+  const uint32_t sum = c0 + c1;
+  const uint32_t above = block_excl_scan(sum, warp_tot, total);
+  if (above < krem && krem <= above + sum) {
+    if (krem <= above + c0) {
+      *digit = static_cast<uint32_t>(nb - 1 - tid * per);
+      *krem_out = krem - above;
+    } else {
+      *digit = static_cast<uint32_t>(nb - 2 - tid * per);
+      *krem_out = krem - above - c0;
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(TG_THREADS, 1)
+    topk_threshold_kernel(int64_t n_free, int64_t k_free, TopkScratch t, float *__restrict__ kth_out) {
+  __shared__ uint32_t h[TG_BINS];
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t s_total, s_digit, s_krem;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  uint32_t T = 0xFFFFFFFFu, need_eq = 0u;
+  if (k_free > 0) {
+    for (int b = tid; b < TG_BINS; b += TG_THREADS) h[b] = t.hist[b];
+    __syncthreads();
+    tg_find_bin(h, TG_BINS, static_cast<uint32_t>(k_free), warp_tot, &s_total, &s_digit, &s_krem);
+    uint32_t prefix = s_digit << 21, mask = 0x7FFu << 21, krem = s_krem;
+    // two more digits: bits [20, 10) and [9, 0)
+    for (int d = 0; d < 2; ++d) {
+      const int shift = d == 0 ? 10 : 0;
+      const int nb = d == 0 ? 2048 : 1024;
+      for (int b = tid; b < TG_BINS; b += TG_THREADS) h[b] = 0u;
+      __syncthreads();
+      // eight loads in flight per thread: one CTA streams all keys from L2
+      for (int64_t base = 0; base < n_free; base += TG_THREADS * TG_LOADS) {
+        uint32_t kv[TG_LOADS];
+#pragma unroll
+        for (int q = 0; q < TG_LOADS; ++q) {
+          const int64_t i = base + q * TG_THREADS + tid;
+          kv[q] = i < n_free ? __ldcg(t.keys + i) : ~prefix;  // ~prefix never matches
+        }
+#pragma unroll
+        for (int q = 0; q < TG_LOADS; ++q)
+          warp_hist_add(h, (kv[q] >> shift) & static_cast<uint32_t>(nb - 1), (kv[q] & mask) == prefix);
+      }
+      __syncthreads();
+      tg_find_bin(h, nb, krem, warp_tot, &s_total, &s_digit, &s_krem);
+      prefix |= s_digit << shift;
+      mask |= static_cast<uint32_t>(nb - 1) << shift;
+      krem = s_krem;
+    }
+    T = prefix;
+    need_eq = krem;
+  }
+  if (tid == 0) {
+    t.sel[0] = T;
+    t.sel[1] = need_eq;
+    if (kth_out) *kth_out = k_free > 0 ? key_value(T) : __uint_as_float(0x7FC00000u);
+  }
+}
+
+// Per chunk: keys > T and == T (chunk c = keys [c chunk2, (c + 1) chunk2)).
+__global__ void __launch_bounds__(TG_THREADS)
+    topk_count_kernel(int64_t n_free, int64_t chunk2, TopkScratch t) {
+  __shared__ uint32_t red[2][32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const uint32_t T = t.sel[0];
+  const int64_t i0 = blockIdx.x * chunk2, i1 = min(n_free, i0 + chunk2);
+  uint32_t gt = 0, eq = 0;
+  for (int64_t i = i0 + tid; i < i1; i += TG_THREADS) {
+    const uint32_t key = t.keys[i];
+    gt += key > T;
+    eq += key == T;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gt += __shfl_xor_sync(0xffffffffu, gt, o);
+    eq += __shfl_xor_sync(0xffffffffu, eq, o);
+  }
+  if (lane == 0) {
+    red[0][w] = gt;
+    red[1][w] = eq;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int k = 1; k < 32; ++k) {
+      gt += red[0][k];
+      eq += red[1][k];
+    }
+    t.chunk[blockIdx.x] = gt;
+    t.chunk[TG_MAX_CTAS + blockIdx.x] = eq;
+  }
+}
+
+constexpr int TG_ITEMS = 2;
+
+__global__ void __launch_bounds__(TG_THREADS)
+    topk_write_kernel(int64_t n_free, int64_t k_free, int64_t tail, int64_t chunk2, TopkScratch t,
+                      int32_t *__restrict__ idx_out) {
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t s_total;
+  const int tid = threadIdx.x;
+  if (blockIdx.x == 0)
+    for (int64_t q = tid; q < tail; q += TG_THREADS) idx_out[k_free + q] = static_cast<int32_t>(n_free + q);
+  if (k_free == 0) return;
+  const uint32_t T = t.sel[0], need_eq = t.sel[1];
+  // keys > T and == T in the chunks before this one
+  __shared__ uint32_t s_before[2];
+  if (tid < 32) {
+    uint32_t g = 0, e = 0;
+    for (int c = tid; c < static_cast<int>(blockIdx.x); c += 32) {
+      g += t.chunk[c];
+      e += t.chunk[TG_MAX_CTAS + c];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      g += __shfl_xor_sync(0xffffffffu, g, o);
+      e += __shfl_xor_sync(0xffffffffu, e, o);
+    }
+    if (tid == 0) {
+      s_before[0] = g;
+      s_before[1] = e;
+    }
+  }
+  __syncthreads();
+  uint32_t run_gt = s_before[0], run_eq = s_before[1];
+  const int64_t i0 = blockIdx.x * chunk2, i1 = min(n_free, i0 + chunk2);
+  for (int64_t base = i0; base < i1; base += static_cast<int64_t>(TG_THREADS) * TG_ITEMS) {
+    const int64_t j0 = base + static_cast<int64_t>(tid) * TG_ITEMS;
+    uint32_t kk[TG_ITEMS];
+    uint32_t ngt = 0, neq = 0;
+#pragma unroll
+    for (int q = 0; q < TG_ITEMS; ++q) {
+      const int64_t i = j0 + q;
+      kk[q] = i < i1 ? t.keys[i] : 0u;
+      if (i < i1) {
+        ngt += kk[q] > T;
+        neq += kk[q] == T;
+      }
+    }
+    const uint32_t excl = block_excl_scan(ngt | (neq << 16), warp_tot, &s_total);
+    uint32_t gt_before = run_gt + (excl & 0xFFFFu);
+    uint32_t eq_before = run_eq + (excl >> 16);
+#pragma unroll
+    for (int q = 0; q < TG_ITEMS; ++q) {
+      const int64_t i = j0 + q;
+      if (i >= i1) break;
+      if (kk[q] > T) {
+        idx_out[gt_before + min(eq_before, need_eq)] = static_cast<int32_t>(i);
+        ++gt_before;
+      } else if (kk[q] == T) {
+        if (eq_before < need_eq) idx_out[gt_before + eq_before] = static_cast<int32_t>(i);
+        ++eq_before;
+      }
+    }
+    run_gt += s_total & 0xFFFFu;
+    run_eq += s_total >> 16;
+    __syncthreads();
+  }
+}
+
+size_t topk_scratch_bytes(int64_t Nc) {
+  return tg_round(static_cast<size_t>(Nc > 0 ? Nc : 1) * 4) + tg_round(TG_BINS * 4) + tg_round(2 * TG_MAX_CTAS * 4) +
+         tg_round(4 * TG_MAX_CTAS * 4) + 256;
+}
+
 spts_status launch_select_topk(const float *s_a, const float *s_b, int mode, float w_a, float w_b, int64_t Nc,
                                int64_t k, int64_t force_tail, int32_t *idx_out, float *fused_out,
-                               float *kth_out, uint32_t *status, cudaStream_t s) {
+                               float *kth_out, uint32_t *status, void *scratch, cudaStream_t s) {
   FuseArgs fa{s_a, s_b, mode, w_a, w_b, 0.f, 0.f};
   const int64_t n_free = Nc - force_tail;
+  if (scratch != nullptr && n_free > TK_GRID_MIN) {
+    const TopkScratch t = tg_carve(scratch, n_free);
+    const int64_t want = (Nc + TG_THREADS - 1) / TG_THREADS;
+    const int n_cta = static_cast<int>(std::min<int64_t>(std::min(num_sms(), TG_MAX_CTAS), want));
+    const int64_t chunk = (Nc + n_cta - 1) / n_cta;
+    const int64_t chunk2 = (n_free + n_cta - 1) / n_cta;
+    topk_prep_kernel<<<n_cta, TG_THREADS, 0, s>>>(fa, Nc, chunk, t);
+    note_launch();
+    topk_keys_kernel<<<n_cta, TG_THREADS, 0, s>>>(fa, Nc, n_free, chunk, n_cta, t, fused_out, status);
+    note_launch();
+    topk_threshold_kernel<<<1, TG_THREADS, 0, s>>>(n_free, k - force_tail, t, kth_out);
+    note_launch();
+    if (k > force_tail) {
+      topk_count_kernel<<<n_cta, TG_THREADS, 0, s>>>(n_free, chunk2, t);
+      note_launch();
+    }
+    topk_write_kernel<<<n_cta, TG_THREADS, 0, s>>>(n_free, k - force_tail, force_tail, chunk2, t, idx_out);
+    note_launch();
+    SPTS_CUDA_TRY(cudaGetLastError());
+    return SPTS_OK;
+  }
   if (n_free <= TK_SMEM_KEYS) {
     const size_t smem = static_cast<size_t>(n_free > 0 ? n_free : 1) * sizeof(uint32_t);
     static bool attr = false;
