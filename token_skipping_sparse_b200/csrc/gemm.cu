@@ -97,22 +97,23 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
     const int32_t pos = live ? p.row_pos[row] : 0;
 #pragma unroll 1
-    for (int hc = 0; hc < BN / 128; ++hc) {     // heads of 128 columns in this tile
+    for (int c = 0; c < 2; ++c) {               // pairs i in [32c, 32c+32), partner i+64
+      // one angle per pair, shared by the tile's heads (same row position)
+      float cs[32], sn[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) rope_angle_f(pos, p.freqs.inv_freq[c * 32 + i], &cs[i], &sn[i]);
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {             // pairs i in [32c, 32c+32), partner i+64
+      for (int hc = 0; hc < BN / 128; ++hc) {   // heads of 128 columns in this tile
         uint32_t lo[32], hi[32];
         tmem_ld32(tbase + hc * 128 + c * 32, lo);
         tmem_ld32(tbase + hc * 128 + 64 + c * 32, hi);
         tmem_ld_wait();
-        float *xl = reinterpret_cast<float *>(lo);
-        float *xh = reinterpret_cast<float *>(hi);
         float yl[32], yh[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          float cs, sn;
-          rope_angle_f(pos, p.freqs.inv_freq[c * 32 + i], &cs, &sn);
-          yl[i] = xl[i] * cs - xh[i] * sn;
-          yh[i] = xh[i] * cs + xl[i] * sn;
+          const float xl = __uint_as_float(lo[i]), xh = __uint_as_float(hi[i]);
+          yl[i] = xl * cs[i] - xh * sn[i];
+          yh[i] = xh * cs[i] + xl * sn[i];
         }
         if (live) {
           __nv_bfloat16 *o = out + row * p.N + tn * BN + hc * 128;
@@ -134,7 +135,8 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
       for (int i = 0; i < 32; ++i) y[i] = silu(__uint_as_float(g[i])) * __uint_as_float(u[i]);
       if (live) store_bf16x32(out + row * p.N + tn * 128 + c * 32, y);
     }
-  } else {  // SCATTER_ADD into fp32 rows
+  } else {  // SCATTER_ADD into fp32 rows: rows are unique, so one vector reduction per 4 columns
+           // performs the single fp32 add h + acc in L2 without a load round trip
     float *out = static_cast<float *>(p.out);
     const int64_t orow = live ? p.rows[row] : 0;
 #pragma unroll 1
@@ -143,16 +145,12 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
       tmem_ld32(tbase + c * 32, r);
       tmem_ld_wait();
       if (live) {
-        float4 *dst = reinterpret_cast<float4 *>(out + orow * p.N + tn * BN + c * 32);
+        float *dst = out + orow * p.N + tn * BN + c * 32;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float4 h = dst[q];
-          h.x += __uint_as_float(r[4 * q + 0]);
-          h.y += __uint_as_float(r[4 * q + 1]);
-          h.z += __uint_as_float(r[4 * q + 2]);
-          h.w += __uint_as_float(r[4 * q + 3]);
-          dst[q] = h;
-        }
+        for (int q = 0; q < 8; ++q)
+          asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * q), "r"(r[4 * q + 0]),
+                       "r"(r[4 * q + 1]), "r"(r[4 * q + 2]), "r"(r[4 * q + 3])
+                       : "memory");
       }
     }
   }
