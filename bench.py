@@ -63,11 +63,14 @@ def layer_work(wl, Nc, k, P, idx_attn, ffn=True):
     i + 1 keys; attention counts only those (causal) pairs.  The probe is
     counted twice (row statistics, then column sums)."""
     D, Hq, Hkv, d, F, r = wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r
-    vis = float(np.sum(idx_attn.astype(np.float64) + 1.0))
+    d_low = wl.ltp_dout or D
+    kv_act = bool(wl.kv_active)
+    # active-row keys only: the t-th selected query sees the t + 1 selected keys
+    vis = k * (k + 1) / 2.0 if kv_act else float(np.sum(idx_attn.astype(np.float64) + 1.0))
     probe_vis = float(sum(Nc - P + p + 1 for p in range(P)))
     fl = {
         "k_proj_rope": 2.0 * Nc * D * Hkv * d,
-        "v_proj": 2.0 * Nc * D * Hkv * d,
+        "v_proj": 2.0 * (k if kv_act else Nc) * D * Hkv * d,
         "probe_q_proj": 2.0 * P * D * Hq * d,
         "probe_scores": 2.0 * (2.0 * Hq * d * probe_vis),
         "q_proj_rope": 2.0 * k * D * Hq * d,
@@ -75,12 +78,13 @@ def layer_work(wl, Nc, k, P, idx_attn, ffn=True):
         "o_proj_scatter": 2.0 * k * Hq * d * D,
     }
     if ffn:
-        fl.update({"ltp_scores": 2.0 * Nc * (D * r + r * D), "gate_up_swiglu": 4.0 * k * D * F,
+        fl.update({"ltp_scores": 2.0 * Nc * (D * r + r * d_low), "gate_up_swiglu": 4.0 * k * D * F,
                    "down_proj_scatter": 2.0 * k * F * D})
-    w_bytes = 2.0 * (D * Hq * d * 2 + D * Hkv * d * 2 + (3 * D * F + 2 * D * r if ffn else 0))
+    w_bytes = 2.0 * (D * Hq * d * 2 + D * Hkv * d * 2 + (3 * D * F + D * r + r * d_low if ffn else 0))
+    kv_rows = (Nc + 2 * k) if kv_act else 2 * Nc             # K (+ gathered K_sel and V_sel) or K and V
     act_bytes = (Nc * D * 4 * 2 * (2 if ffn else 1)          # h read by each norm, written back
                  + Nc * D * 2 * 2 * (2 if ffn else 1)        # normed rows written and read
-                 + Nc * Hkv * d * 2 * 2 * 2                  # K, V written and read
+                 + kv_rows * Hkv * d * 2 * 2                 # K, V written and read
                  + k * Hq * d * 2 * 4                        # Q_sel and O_sel written and read
                  + (k * F * 2 * 2 if ffn else 0))            # SwiGLU activation written and read
     return fl, w_bytes + act_bytes
@@ -163,7 +167,8 @@ class LayerCase:
         wl = self.wl
         return self.S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k if k is None else k,
                                  fuse=wl.fuse, salient_rows=self.sal if len(self.sal) else None,
-                                 salient_shift=wl.salient_shift)
+                                 salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout,
+                                 kv_active_only=wl.kv_active)
 
 
 def run_msdp_step(S, wl, h, pos, layers, desc):
@@ -415,7 +420,10 @@ def oracle_baseline(inp, row_sample=1024, sel_sample=16):
     t2 = time.perf_counter()
     xr = O.bf16_round(O.rmsnorm(h[rows], None, 1e-5))
     qs = O.bf16_round(O.rope((xr @ W["w_q"].T).reshape(len(rows), Hq, d), pos[rows]))
-    o = O.bf16_round(O.reduced_attention(qs, pos[rows], kk, inp.vv, pos))
+    if wl.kv_active:  # keys and values of the selected rows only
+        o = O.bf16_round(O.reduced_attention(qs, pos[rows], kk[idx], inp.vv[idx], pos[idx]))
+    else:
+        o = O.bf16_round(O.reduced_attention(qs, pos[rows], kk, inp.vv, pos))
     h1 = h[rows] + o.reshape(len(rows), -1) @ W["w_o"].T
     if wl.F:
         O.reduced_ffn(h1, np.arange(len(rows)), None, 1e-5, W["w_gate"], W["w_up"], W["w_down"])
@@ -461,7 +469,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.steps is None:
-        args.steps = DEFAULT_STEPS.get(args.workload, 50) if args.impl == "ours" else 3
+        base = args.workload.rsplit("_", 1)[0]  # a variant takes its base workload's count
+        args.steps = (DEFAULT_STEPS.get(args.workload, DEFAULT_STEPS.get(base, 50)) if args.impl == "ours" else 3)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))

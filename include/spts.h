@@ -280,6 +280,13 @@ typedef struct {
   const int32_t *salient_rows;
   int64_t n_salient;
   float salient_shift;
+  /* LTP proxy output channels: B is [ltp_dout, r] (the channel-reduced
+   * proxy D_low of Table A); 0 means D.                                    */
+  int ltp_dout;
+  /* 1: the reduced attention uses the keys and values of the active rows
+   * only (K and V of idx_attn), the KV-cache reading behind Table 5; V is
+   * then projected for the active rows only.  0: all Nc candidate keys.   */
+  int kv_active_only;
 } spts_layer_desc;
 
 typedef struct {

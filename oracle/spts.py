@@ -323,6 +323,7 @@ class LayerConfig:
     theta: float = 500000.0
     salient_rows: np.ndarray | None = None   # workload recipe, not SPTS
     salient_shift: float = 0.0
+    kv_active: bool = False    # reduced attention over the active rows' keys only
 
 
 def inject_salience(kk, q_probe, rows, shift, Hkv):
@@ -365,7 +366,13 @@ def layer_forward(h, pos, W: LayerWeights, cfg: LayerConfig, trace: dict | None 
     s32 = s.astype(np.float32)
     idx_a, tau_a = select_topk(s32, k, P)
     q_sel = bf16_round(rope((xn[idx_a] @ W.w_q.T).reshape(k, Hq, d), pos[idx_a], cfg.theta))
-    o_sel = bf16_round(reduced_attention(q_sel, pos[idx_a], kk, vv, pos))
+    if cfg.kv_active:
+        # the KV-cache reading behind Table 5 and Fig. A(c): a skipping layer
+        # keeps K and V of its active tokens only, so the selected queries
+        # attend, causally by original position, to the selected keys
+        o_sel = bf16_round(reduced_attention(q_sel, pos[idx_a], kk[idx_a], vv[idx_a], pos[idx_a]))
+    else:
+        o_sel = bf16_round(reduced_attention(q_sel, pos[idx_a], kk, vv, pos))
     h1 = attention_residual(h, idx_a, o_sel, W.w_o)
     t.update(xn=xn, k=kk, v=vv, q_probe=q_probe, s=s, group=group, idx_attn=idx_a,
              tau_attn=tau_a, q_sel=q_sel, o_sel=o_sel, h_attn=h1)

@@ -45,6 +45,8 @@ class Workload:
     layers: int = 1
     ratios: tuple = ()
     seed: int = 1000
+    ltp_dout: int = 0         # LTP proxy output channels (0: D)
+    kv_active: bool = False   # reduced attention over the active rows' keys only
 
     @property
     def k(self) -> int:
@@ -78,6 +80,18 @@ WORKLOADS = {
     "msdp_small": Workload("msdp_small", N=600, Hq=8, Hkv=2, d=128, P=16, keep="0.8", D=1024,
                            F=1024, r=64, layers=8, ratios=("0.8", "0.6", "0.4", "0.25"), seed=1102),
 }
+# Variants of the layer workloads (the same inputs, one setting changed):
+#   _kv    keys and values of the active rows only in the reduced attention;
+#   _mul   the Multiply fusion f = s * c for the FFN selection;
+#   _p1    a single probe token;
+#   _dlow  the channel-reduced LTP proxy, D_low = 512 output channels, r = 192.
+for _base in ("layer_32k", "layer_128k", "layer_small"):
+    _w = WORKLOADS[_base]
+    WORKLOADS[_base + "_kv"] = replace(_w, name=_base + "_kv", kv_active=True)
+    WORKLOADS[_base + "_mul"] = replace(_w, name=_base + "_mul", fuse=FUSE_MULTIPLY)
+    WORKLOADS[_base + "_p1"] = replace(_w, name=_base + "_p1", P=1)
+    WORKLOADS[_base + "_dlow"] = replace(_w, name=_base + "_dlow", ltp_dout=512, r=192)
+del _base, _w
 
 
 def _gen(seed):
@@ -129,7 +143,8 @@ def make_layer_weights(wl: Workload, layer: int = 0):
     """bf16 weights of one Llama-shaped layer, nn.Linear layout, ~N(0, 0.02).
 
     Keys: w_q [Hq*d, D], w_k / w_v [Hkv*d, D], w_o [D, Hq*d]; when F > 0 also
-    w_gate / w_up [F, D], w_down [D, F], ltp_a [r, D], ltp_b [D, r].  Norm
+    w_gate / w_up [F, D], w_down [D, F], ltp_a [r, D], ltp_b [D_low, r] (D_low =
+    ltp_dout, else D).  Norm
     weights are ones.
     """
     g = _gen(wl.seed * 1000 + 17 + 101 * layer)
@@ -141,7 +156,7 @@ def make_layer_weights(wl: Workload, layer: int = 0):
     out = dict(w_q=w(hd, D), w_k=w(kd, D), w_v=w(kd, D), w_o=w(D, hd))
     if wl.F:
         out.update(w_gate=w(wl.F, D), w_up=w(wl.F, D), w_down=w(D, wl.F),
-                   ltp_a=w(wl.r, D), ltp_b=w(D, wl.r))
+                   ltp_a=w(wl.r, D), ltp_b=w(wl.ltp_dout or D, wl.r))
     out["norm_attn"] = torch.ones(D, dtype=torch.bfloat16)
     out["norm_ffn"] = torch.ones(D, dtype=torch.bfloat16)
     return out

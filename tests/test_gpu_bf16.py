@@ -37,7 +37,7 @@ def test_reduced_attention_bf16(Nc, k, Hq, Hkv):
 
 
 @pytest.mark.parametrize("Nc,P,Hq,Hkv", [(1000, 16, 8, 2), (3000, 64, 32, 8), (2000, 128, 32, 8), (300, 64, 8, 8),
-                                         (700, 20, 8, 4), (2500, 80, 32, 8), (130, 100, 32, 8)])
+                                         (700, 20, 8, 4), (2500, 80, 32, 8), (130, 100, 32, 8), (1000, 1, 32, 8)])
 def test_probe_scores_bf16(Nc, P, Hq, Hkv):
     pos = _positions(Nc)
     q = torch.randn(P, Hq, 128).to(torch.bfloat16)
@@ -51,7 +51,8 @@ def test_probe_scores_bf16(Nc, P, Hq, Hkv):
     assert abs(float(s.double().sum()) - P * Hq) < 1e-3 * P * Hq
 
 
-@pytest.mark.parametrize("Nc,D,r,Dout", [(1000, 1024, 64, 1024), (300, 4096, 256, 4096), (129, 512, 128, 768)])
+@pytest.mark.parametrize("Nc,D,r,Dout", [(1000, 1024, 64, 1024), (300, 4096, 256, 4096), (129, 512, 128, 768),
+                                         (700, 4096, 192, 512)])
 def test_ltp_scores_bf16(Nc, D, r, Dout):
     x = torch.randn(Nc, D).to(torch.bfloat16)
     A = (0.02 * torch.randn(r, D)).to(torch.bfloat16)
@@ -71,17 +72,22 @@ def _layer_case(name):
     return wl, h, W, sal, pos
 
 
-def test_layer_small_matches_oracle():
-    wl, h, W, sal, pos = _layer_case("layer_small")
+# the base layer and its variants: active-row keys only, Multiply fusion, one
+# probe token, the channel-reduced LTP proxy
+@pytest.mark.parametrize("name", ["layer_small", "layer_small_kv", "layer_small_mul", "layer_small_p1",
+                                  "layer_small_dlow"])
+def test_layer_small_matches_oracle(name):
+    wl, h, W, sal, pos = _layer_case(name)
     Wd = {n: t.cuda() for n, t in W.items()}
     desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k, fuse=wl.fuse,
-                        salient_rows=sal.cuda(), salient_shift=wl.salient_shift)
+                        salient_rows=sal.cuda(), salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout,
+                        kv_active_only=wl.kv_active)
     hd = h.cuda()
     out = S.spts_layer_forward(hd, pos.cuda(), desc, Wd, outputs=True)
     S.check_device_status()
     ow = O.LayerWeights(**{n: np64(t) for n, t in W.items()})
     cfg = O.LayerConfig(Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, P=wl.P, k=wl.k, fuse=wl.fuse,
-                        salient_rows=sal.numpy(), salient_shift=wl.salient_shift)
+                        salient_rows=sal.numpy(), salient_shift=wl.salient_shift, kv_active=wl.kv_active)
     tr = {}
     O.layer_forward(np64(h), pos.numpy(), ow, cfg, tr)
     s = out["s"].cpu().numpy()
@@ -89,15 +95,30 @@ def test_layer_small_matches_oracle():
     ia = out["idx_attn"].cpu().numpy()
     band_check(ia, tr["idx_attn"], tr["s"], tr["tau_attn"])
     # reduced attention rows: oracle computes every row, compare at the GPU's picks
-    q_all = O.bf16_round(O.rope((tr["xn"] @ ow.w_q.T).reshape(wl.N, wl.Hq, wl.d), pos.numpy()))
-    o_all = O.bf16_round(O.reduced_attention(q_all, pos.numpy(), tr["k"], tr["v"], pos.numpy()))
-    assert_bf16_close(np64(out["o_sel"]), o_all[ia], 2e-2, "o_sel")
+    pn = pos.numpy()
+    q_all = O.bf16_round(O.rope((tr["xn"] @ ow.w_q.T).reshape(wl.N, wl.Hq, wl.d), pn))
+    if wl.kv_active:  # the keys are the GPU's active rows
+        o_sel = O.bf16_round(O.reduced_attention(q_all[ia], pn[ia], tr["k"][ia], tr["v"][ia], pn[ia]))
+    else:
+        o_sel = O.bf16_round(O.reduced_attention(q_all, pn, tr["k"], tr["v"], pn))[ia]
+    assert_bf16_close(np64(out["o_sel"]), o_sel, 2e-2, "o_sel")
+    ha = np64(out["h_attn"])
     same = np.array_equal(ia, tr["idx_attn"])
     if same:
-        assert_close(np64(out["h_attn"]), tr["h_attn"], 2e-2, "h after attention")
-        c = out["c"].cpu().numpy()
-        assert_close(c, tr["c"], 1e-3 * tr["c"].max(), "ltp scores")
-        idf = out["idx_ffn"].cpu().numpy()
-        band_check(idf, tr["idx_ffn"], tr["f"], tr["tau_ffn"])
-        if np.array_equal(idf, tr["idx_ffn"]):
-            assert_close(np64(hd), tr["h_out"], 2e-2, "h out")
+        assert_close(ha, tr["h_attn"], 2e-2, "h after attention")
+    # a8-a10 from the GPU's own h' (each step checked on the same input): LTP
+    # within the per-call bound, then the fused score and the FFN set exactly
+    # (the same fp32 operations on the same scores), then the reduced FFN
+    x2 = O.bf16_round(O.rmsnorm(ha, ow.norm_ffn, cfg.eps))
+    c_want = O.ltp_scores(x2, ow.ltp_a, ow.ltp_b)
+    c = out["c"].cpu().numpy()
+    assert_close(c, c_want, 1e-3 * c_want.max(), "ltp scores")
+    f_want = O.fuse_scores(s.astype(np.float32), c.astype(np.float32), wl.fuse, 0.5, 0.5)
+    assert np.array_equal(out["f"].cpu().numpy().view(np.uint32), f_want.view(np.uint32)), "fused score"
+    idf = out["idx_ffn"].cpu().numpy()
+    assert np.array_equal(idf, O.select_topk(f_want, wl.k, wl.P)[0]), "FFN selection"
+    h_want = O.reduced_ffn(ha, idf, ow.norm_ffn, cfg.eps, ow.w_gate, ow.w_up, ow.w_down)
+    assert_close(np64(hd), h_want, 2e-2, "h out (reduced FFN on the GPU's h')")
+    # the composed layer against the oracle's own chain: two bf16-stored stages
+    if same and np.array_equal(idf, tr["idx_ffn"]):
+        assert_close(np64(hd), tr["h_out"], 4e-2, "h out (composed)")

@@ -68,7 +68,8 @@ def _run_gpu_layer(wl, h, W, pos, sal, k=None):
     Wd = {n: t.cuda() for n, t in W.items()}
     sal_d = sal.cuda() if len(sal) else None
     desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k if k is None else k, fuse=wl.fuse,
-                        salient_rows=sal_d, salient_shift=wl.salient_shift)
+                        salient_rows=sal_d, salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout,
+                        kv_active_only=wl.kv_active)
     hd = h.cuda()
     out = S.spts_layer_forward(hd, pos.cuda(), desc, Wd, outputs=True)
     S.check_device_status()
@@ -105,7 +106,9 @@ def _check_layer_sampled(wl, h, W, pos, sal, g, k, n_rows=40):
     rows = ia[pick]
     q = O.bf16_round(O.rope((xn[rows].astype(np.float64) @ Wn["w_q"].T).reshape(len(rows), wl.Hq, wl.d),
                             pos_n[rows]))
-    o = O.bf16_round(O.reduced_attention(q, pos_n[rows], K, V, pos_n))
+    # the keys: every candidate, or (kv_active) the GPU's active rows
+    Kk, Vk, pk = (K[ia], V[ia], pos_n[ia]) if wl.kv_active else (K, V, pos_n)
+    o = O.bf16_round(O.reduced_attention(q, pos_n[rows], Kk, Vk, pk))
     assert_bf16_close(np64(g["o_sel"][pick]), o, 2e-2, "o_sel rows")
     h1_rows = h64[rows] + o.reshape(len(rows), -1) @ Wn["w_o"].T
     ha = g["h_attn"].numpy()
@@ -123,7 +126,7 @@ def _check_layer_sampled(wl, h, W, pos, sal, g, k, n_rows=40):
             rs = rr[sel]
             qq = O.bf16_round(O.rope((xn[rs].astype(np.float64) @ Wn["w_q"].T).reshape(len(rs), wl.Hq, wl.d),
                                      pos_n[rs]))
-            oo = O.bf16_round(O.reduced_attention(qq, pos_n[rs], K, V, pos_n))
+            oo = O.bf16_round(O.reduced_attention(qq, pos_n[rs], Kk, Vk, pk))
             out[sel] += oo.reshape(len(rs), -1) @ Wn["w_o"].T
         return out
 
@@ -150,7 +153,8 @@ def _check_layer_sampled(wl, h, W, pos, sal, g, k, n_rows=40):
     assert len(fsel) > 0
 
 
-@pytest.mark.parametrize("name", ["attn_8k", "layer_32k", "layer_128k"])
+@pytest.mark.parametrize("name", ["attn_8k", "layer_32k", "layer_128k", "layer_32k_kv", "layer_128k_kv",
+                                  "layer_32k_mul", "layer_32k_dlow"])
 def test_layer_full_size_sampled(name):
     wl = WORKLOADS[name]
     h = make_hidden(wl)

@@ -293,6 +293,34 @@ def test_layer_keep_all_equals_dense_layer():
     np.testing.assert_allclose(out, _dense_layer_torch(h, pos, W, cfg), rtol=1e-11, atol=1e-11)
 
 
+
+def test_layer_kv_active_keep_all_equals_dense_layer():
+    # with every row active, the active-row keys are all keys: the dense layer
+    h, pos, W, cfg = _tiny_layer()
+    cfg.kv_active = True
+    out, _ = O.layer_forward(h, pos, W, cfg)
+    np.testing.assert_allclose(out, _dense_layer_torch(h, pos, W, cfg), rtol=1e-11, atol=1e-11)
+
+
+def test_layer_kv_active_attention_is_dense_attention_of_the_active_rows():
+    # with keys restricted to the active rows, each selected query attends as
+    # in a dense causal layer run on the subsequence of the selected rows
+    h, pos, W, cfg = _tiny_layer(N=64, k=21, P=3)
+    cfg.kv_active = True
+    tr = {}
+    O.layer_forward(h, pos, W, cfg, tr)
+    idx = tr["idx_attn"]
+    T = torch.from_numpy
+    Hq, Hkv, d, m = cfg.Hq, cfg.Hkv, cfg.d, len(idx)
+    x = T(tr["xn"][idx])
+    k = O.bf16_round(O.rope(F.linear(x, T(W.w_k)).numpy().reshape(m, Hkv, d), pos[idx]))
+    v = O.bf16_round(F.linear(x, T(W.w_v)).numpy().reshape(m, Hkv, d))
+    kk = np.repeat(k, Hq // Hkv, axis=1).transpose(1, 0, 2).copy()
+    vv = np.repeat(v, Hq // Hkv, axis=1).transpose(1, 0, 2).copy()
+    q = tr["q_sel"].transpose(1, 0, 2).copy()
+    want = F.scaled_dot_product_attention(T(q), T(kk), T(vv), is_causal=True).numpy().transpose(1, 0, 2)
+    np.testing.assert_allclose(tr["o_sel"], O.bf16_round(want), rtol=0, atol=1e-12)
+
 def test_layer_skipped_rows_pass_through():
     h, pos, W, cfg = _tiny_layer(N=64, k=20, P=4)
     tr = {}

@@ -61,7 +61,8 @@ class LayerDesc(C.Structure):
     _fields_ = [("D", C.c_int), ("Hq", C.c_int), ("Hkv", C.c_int), ("d", C.c_int), ("F", C.c_int),
                 ("r", C.c_int), ("P", C.c_int), ("k", C.c_int64), ("fuse", C.c_int), ("w_a", C.c_float),
                 ("w_b", C.c_float), ("eps", C.c_float), ("theta", C.c_double), ("salient_rows", C.c_void_p),
-                ("n_salient", C.c_int64), ("salient_shift", C.c_float)]
+                ("n_salient", C.c_int64), ("salient_shift", C.c_float), ("ltp_dout", C.c_int),
+                ("kv_active_only", C.c_int)]
 
 
 class LayerWeights(C.Structure):
@@ -325,10 +326,11 @@ def spts_inject_salience(k, q_probe, rows, shift):
 
 # ---------------------------------------------------------------- the composed layer
 def layer_desc(D, Hq, Hkv, d, F, r, P, k, fuse=FUSE_MAXNORM_ADD, w_a=0.5, w_b=0.5, eps=1e-5, theta=500000.0,
-               salient_rows=None, salient_shift=0.0):
+               salient_rows=None, salient_shift=0.0, ltp_dout=0, kv_active_only=False):
     n_sal = 0 if salient_rows is None else int(salient_rows.numel())
     desc = LayerDesc(D, Hq, Hkv, d, F, r, P, k, fuse, w_a, w_b, eps, theta,
-                     None if n_sal == 0 else salient_rows.data_ptr(), n_sal, salient_shift)
+                     None if n_sal == 0 else salient_rows.data_ptr(), n_sal, salient_shift, ltp_dout,
+                     1 if kv_active_only else 0)
     desc._keep = salient_rows  # the descriptor holds a raw pointer: keep the tensor alive with it
     return desc
 

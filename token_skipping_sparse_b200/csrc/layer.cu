@@ -16,6 +16,7 @@ struct LayerBufs {
   float *s, *group, *stats, *c, *f;
   int32_t *idx_a, *idx_f, *qpos;
   void *topk;  // scratch of the grid top-k
+  void *ksel;  // K of the active rows (kv_active_only)
 };
 
 // Carves the workspace; with cv.base == nullptr it only measures.
@@ -39,6 +40,7 @@ void carve(Carver &cv, const spts_layer_desc *L, int64_t Nc, LayerBufs &b) {
   b.idx_f = static_cast<int32_t *>(cv.take(k * 4));
   b.qpos = static_cast<int32_t *>(cv.take(k * 4));
   b.topk = cv.take(topk_scratch_bytes(Nc));
+  b.ksel = cv.take(k * hk * 2);
 }
 
 // A side stream and fork/join events per (host thread, device): the V and
@@ -84,7 +86,11 @@ spts_status check_layer(const spts_layer_desc *L, const spts_layer_weights *W, i
                  "%s: FFN / LTP weights missing", who);
     SPTS_REQUIRE(L->fuse >= SPTS_FUSE_NONE && L->fuse <= SPTS_FUSE_MULTIPLY, SPTS_ERR_INVALID, "%s: bad fusion",
                  who);
+    SPTS_REQUIRE(L->ltp_dout == 0 || (L->ltp_dout > 0 && L->ltp_dout % 256 == 0), SPTS_ERR_SHAPE,
+                 "%s: ltp_dout must be 0 (= D) or a multiple of 256", who);
   }
+  SPTS_REQUIRE(L->kv_active_only == 0 || L->kv_active_only == 1, SPTS_ERR_INVALID, "%s: kv_active_only is 0 or 1",
+               who);
   SPTS_REQUIRE(L->n_salient == 0 || L->salient_rows != nullptr, SPTS_ERR_INVALID, "%s: salient rows NULL", who);
   return SPTS_OK;
 }
@@ -150,18 +156,19 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   const void *xtail = static_cast<const char *>(b.xn) + static_cast<size_t>(Nc - P) * D * 2;
   GemmArgs gq{xtail, P, D, W->w_q, nullptr, hq, SPTS_EPI_ROPE, b.qprobe, nullptr, pos + (Nc - P), L->theta, st};
   GemmArgs gv{b.xn, Nc, D, W->w_v, nullptr, hk, SPTS_EPI_STORE, b.vv, nullptr, nullptr, 0.0, st};
+  const bool kv_active = L->kv_active_only != 0;  // V only for the active rows, later
   if (side) {  // fork: probe-Q and V projections on the side stream
     SPTS_CUDA_TRY(cudaEventRecord(side->fork, s));
     SPTS_CUDA_TRY(cudaStreamWaitEvent(side->s, side->fork, 0));
     SPTS_TRY(launch_gemm(gq, side->s));
     SPTS_CUDA_TRY(cudaEventRecord(side->qprobe_done, side->s));
-    SPTS_TRY(launch_gemm(gv, side->s));
+    if (!kv_active) SPTS_TRY(launch_gemm(gv, side->s));
     SPTS_CUDA_TRY(cudaEventRecord(side->v_done, side->s));
   }
   GemmArgs gk{b.xn, Nc, D, W->w_k, nullptr, hk, SPTS_EPI_ROPE, b.kk, nullptr, pos, L->theta, st};
   SPTS_TRY(launch_gemm(gk, s));
   SPTS_TRY(mark(2));
-  if (!side) SPTS_TRY(launch_gemm(gv, s));
+  if (!side && !kv_active) SPTS_TRY(launch_gemm(gv, s));
   SPTS_TRY(mark(3));
   if (side) SPTS_CUDA_TRY(cudaStreamWaitEvent(s, side->qprobe_done, 0));
   else SPTS_TRY(launch_gemm(gq, s));
@@ -190,7 +197,16 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
     SPTS_CUDA_TRY(cudaStreamWaitEvent(s, side->v_done, 0));
     guard.joined = true;
   }
-  SPTS_TRY(launch_attention_bf16(b.qsel, b.qpos, k, b.kk, b.vv, pos, Nc, L->Hq, L->Hkv, scale, osel, st, s));
+  if (kv_active) {
+    // keys and values of the active rows only: K gathered, V projected from
+    // the gathered normalised rows, key positions = the active positions
+    SPTS_TRY(launch_gather_rows(b.kk, Nc, idx_a, k, static_cast<int64_t>(hk) * 2, b.ksel, nullptr, nullptr, st, s));
+    GemmArgs gvs{b.xsel, k, D, W->w_v, nullptr, hk, SPTS_EPI_STORE, b.vv, nullptr, nullptr, 0.0, st};
+    SPTS_TRY(launch_gemm(gvs, s));
+    SPTS_TRY(launch_attention_bf16(b.qsel, b.qpos, k, b.ksel, b.vv, b.qpos, k, L->Hq, L->Hkv, scale, osel, st, s));
+  } else {
+    SPTS_TRY(launch_attention_bf16(b.qsel, b.qpos, k, b.kk, b.vv, pos, Nc, L->Hq, L->Hkv, scale, osel, st, s));
+  }
   SPTS_TRY(mark(9));
   GemmArgs go{osel, k, hq, W->w_o, nullptr, D, SPTS_EPI_SCATTER_ADD, h, idx_a, nullptr, 0.0, st};
   SPTS_TRY(launch_gemm(go, s));
@@ -207,7 +223,7 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   int32_t *idx_f = o.idx_ffn ? o.idx_ffn : b.idx_f;
   SPTS_TRY(launch_rmsnorm_rows(h, nullptr, Nc, D, W->norm_ffn, L->eps, b.xn, s));
   SPTS_TRY(mark(11));
-  SPTS_TRY(launch_ltp_bf16(b.xn, Nc, D, W->ltp_a, L->r, W->ltp_b, D, c, st, s));
+  SPTS_TRY(launch_ltp_bf16(b.xn, Nc, D, W->ltp_a, L->r, W->ltp_b, L->ltp_dout > 0 ? L->ltp_dout : D, c, st, s));
   SPTS_TRY(mark(12));
   SPTS_TRY(launch_select_topk(sc, c, L->fuse, L->w_a, L->w_b, Nc, k, P, idx_f, f, nullptr, st, b.topk, s));
   SPTS_TRY(launch_gather_rows(b.xn, Nc, idx_f, k, static_cast<int64_t>(D) * 2, b.xsel, nullptr, nullptr, st, s));
