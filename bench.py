@@ -167,7 +167,7 @@ class LayerCase:
         wl = self.wl
         return self.S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k if k is None else k,
                                  fuse=wl.fuse, salient_rows=self.sal if len(self.sal) else None,
-                                 salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout,
+                                 salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m,
                                  kv_active_only=wl.kv_active)
 
 
@@ -384,7 +384,10 @@ class OracleInputs:
         self.kk = O.bf16_round(O.rope((xn @ self.W["w_k"].T).reshape(N, wl.Hkv, wl.d), self.pos))
         self.vv = O.bf16_round((xn @ self.W["w_v"].T).reshape(N, wl.Hkv, wl.d))
         self.xn_tail = xn[N - P:]
-        self.c = O.ltp_scores(xn, self.W["ltp_a"], self.W["ltp_b"]) if wl.F else None
+        self.c = None
+        if wl.F:
+            self.c = (O.ltp_topm_scores(xn, self.W["ltp_a"], self.W["ltp_b"], wl.ltp_top_m) if wl.ltp_top_m
+                      else O.ltp_scores(xn, self.W["ltp_a"], self.W["ltp_b"]))
 
 
 def oracle_baseline(inp, row_sample=1024, sel_sample=16):
@@ -405,7 +408,11 @@ def oracle_baseline(inp, row_sample=1024, sel_sample=16):
     O.bf16_round(O.rope((xs @ W["w_k"].T).reshape(rs, Hkv, d), pos[:rs]))
     O.bf16_round((xs @ W["w_v"].T).reshape(rs, Hkv, d))
     if wl.F:
-        O.ltp_scores(O.bf16_round(O.rmsnorm(h[:rs], None, 1e-5)), W["ltp_a"], W["ltp_b"])
+        xl = O.bf16_round(O.rmsnorm(h[:rs], None, 1e-5))
+        if wl.ltp_top_m:
+            O.ltp_topm_scores(xl, W["ltp_a"], W["ltp_b"], wl.ltp_top_m)
+        else:
+            O.ltp_scores(xl, W["ltp_a"], W["ltp_b"])
     t_lin = time.perf_counter() - t0
     t1 = time.perf_counter()
     qp = O.bf16_round(O.rope((inp.xn_tail @ W["w_q"].T).reshape(P, Hq, d), pos[N - P:]))

@@ -142,6 +142,18 @@ SPTS_API spts_status spts_ltp_scores(spts_dtype dt, const void *x, int64_t Nc, i
                             spts_stream stream);
 SPTS_API size_t spts_ltp_scores_workspace(int64_t Nc, int D, int r, int Dout);
 
+/* Top-rho channel saliency of the same proxy (Table E with the D_low proxy
+ * of Table A): scores[i] = sum of the top_m largest |y_ij| of
+ * y_i = (x_i A^T) B^T over its Dout = D_low channels (top_m = ceil(rho *
+ * D_low)); ties at the threshold count as often as needed to make top_m.
+ * Same operands and layouts as spts_ltp_scores.
+ * Limits: dt = SPTS_BF16; D % 64 == 0; r % 64 == 0, 64 <= r <= 256;
+ * Dout in {256, 512}; 1 <= top_m <= Dout. */
+SPTS_API spts_status spts_ltp_topm_scores(spts_dtype dt, const void *x, int64_t Nc, int D, const void *A, int r,
+                                          const void *B, int Dout, int top_m, float *scores, void *ws,
+                                          size_t ws_bytes, spts_stream stream);
+SPTS_API size_t spts_ltp_topm_scores_workspace(int64_t Nc, int D, int r, int Dout);
+
 /* Token selection (Fig. 2(a)/(b): the informative tokens).
  * The last force_tail candidates are always kept; the other k - force_tail
  * are the largest fused scores among the first Nc - force_tail, equal scores
@@ -287,6 +299,9 @@ typedef struct {
    * only (K and V of idx_attn), the KV-cache reading behind Table 5; V is
    * then projected for the active rows only.  0: all Nc candidate keys.   */
   int kv_active_only;
+  /* > 0: the LTP score is the top-rho channel saliency, the sum of the
+   * ltp_top_m largest |y| (needs ltp_dout in {256, 512}); 0: ||y||_2.      */
+  int ltp_top_m;
 } spts_layer_desc;
 
 typedef struct {

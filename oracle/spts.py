@@ -39,7 +39,7 @@ import numpy as np
 from .accounting import keep_count
 
 __all__ = [
-    "bf16_round", "rmsnorm", "rope", "probe_scores", "ltp_scores", "fuse_scores",
+    "bf16_round", "rmsnorm", "rope", "probe_scores", "ltp_scores", "ltp_topm_scores", "fuse_scores",
     "select_topk", "reduced_attention", "attention_residual", "reduced_ffn",
     "stage_prune", "inject_salience", "LayerWeights", "LayerConfig", "layer_forward",
     "msdp_forward", "MsdpConfig", "FUSE_NONE", "FUSE_MAXNORM_ADD", "FUSE_MULTIPLY",
@@ -156,6 +156,24 @@ def ltp_scores(x, A, B):
     t = bf16_round(x @ np.asarray(A, dtype=np.float64).T)
     y = t @ np.asarray(B, dtype=np.float64).T
     return np.sqrt(np.sum(y * y, axis=1))
+
+
+def ltp_topm_scores(x, A, B, m):
+    """Top-rho channel saliency of the proxy output (Table E, with D_low of
+    Table A).
+
+    Reading: the proxy predicts the token's change y_i = (x_i A^T) B^T over
+    the D_low output channels; the token's saliency is the sum of its m =
+    ceil(rho * D_low) largest |y_ij|.  The intermediate is bf16-rounded as in
+    ltp_scores.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    t = bf16_round(x @ np.asarray(A, dtype=np.float64).T)
+    y = np.abs(t @ np.asarray(B, dtype=np.float64).T)
+    m = int(m)
+    if not 1 <= m <= y.shape[1]:
+        raise ValueError("need 1 <= m <= D_low")
+    return np.sort(y, axis=1)[:, y.shape[1] - m:].sum(axis=1)
 
 
 # --------------------------------------------------------------------------
@@ -324,6 +342,7 @@ class LayerConfig:
     salient_rows: np.ndarray | None = None   # workload recipe, not SPTS
     salient_shift: float = 0.0
     kv_active: bool = False    # reduced attention over the active rows' keys only
+    ltp_top_m: int = 0         # > 0: LTP saliency = sum of the top m |y| (Table E); 0: L2 norm
 
 
 def inject_salience(kk, q_probe, rows, shift, Hkv):
@@ -379,7 +398,8 @@ def layer_forward(h, pos, W: LayerWeights, cfg: LayerConfig, trace: dict | None 
     if not cfg.ffn:
         return h1, s32
     x_ffn = bf16_round(rmsnorm(h1, W.norm_ffn, cfg.eps))
-    c = ltp_scores(x_ffn, W.ltp_a, W.ltp_b)
+    c = (ltp_topm_scores(x_ffn, W.ltp_a, W.ltp_b, cfg.ltp_top_m) if cfg.ltp_top_m > 0
+         else ltp_scores(x_ffn, W.ltp_a, W.ltp_b))
     f = fuse_scores(s32, c.astype(np.float32), cfg.fuse, cfg.w_a, cfg.w_b)
     idx_f, tau_f = select_topk(f, k, P)
     h2 = reduced_ffn(h1, idx_f, W.norm_ffn, cfg.eps, W.w_gate, W.w_up, W.w_down)

@@ -47,6 +47,7 @@ class Workload:
     seed: int = 1000
     ltp_dout: int = 0         # LTP proxy output channels (0: D)
     kv_active: bool = False   # reduced attention over the active rows' keys only
+    ltp_top_m: int = 0        # LTP saliency = sum of the top m |y| (0: L2 norm)
 
     @property
     def k(self) -> int:
@@ -84,13 +85,15 @@ WORKLOADS = {
 #   _kv    keys and values of the active rows only in the reduced attention;
 #   _mul   the Multiply fusion f = s * c for the FFN selection;
 #   _p1    a single probe token;
-#   _dlow  the channel-reduced LTP proxy, D_low = 512 output channels, r = 192.
+#   _dlow  the channel-reduced LTP proxy, D_low = 512 output channels, r = 192;
+#   _rho   that proxy with top-rho saliency, rho = 0.2: the top 103 of 512 |y|.
 for _base in ("layer_32k", "layer_128k", "layer_small"):
     _w = WORKLOADS[_base]
     WORKLOADS[_base + "_kv"] = replace(_w, name=_base + "_kv", kv_active=True)
     WORKLOADS[_base + "_mul"] = replace(_w, name=_base + "_mul", fuse=FUSE_MULTIPLY)
     WORKLOADS[_base + "_p1"] = replace(_w, name=_base + "_p1", P=1)
     WORKLOADS[_base + "_dlow"] = replace(_w, name=_base + "_dlow", ltp_dout=512, r=192)
+    WORKLOADS[_base + "_rho"] = replace(_w, name=_base + "_rho", ltp_dout=512, r=192, ltp_top_m=103)
 del _base, _w
 
 

@@ -62,6 +62,17 @@ def test_ltp_scores_bf16(Nc, D, r, Dout):
     assert_close(c.cpu().numpy(), want, 1e-3 * want.max(), "ltp scores")
 
 
+@pytest.mark.parametrize("Nc,D,r,Dout,m", [(1000, 1024, 192, 512, 103), (300, 4096, 256, 256, 1),
+                                           (129, 512, 64, 512, 512), (700, 4096, 192, 512, 52)])
+def test_ltp_topm_scores_bf16(Nc, D, r, Dout, m):
+    x = torch.randn(Nc, D).to(torch.bfloat16)
+    A = (0.02 * torch.randn(r, D)).to(torch.bfloat16)
+    B = (0.02 * torch.randn(Dout, r)).to(torch.bfloat16)
+    c = S.spts_ltp_topm_scores(x.cuda(), A.cuda(), B.cuda(), m)
+    want = O.ltp_topm_scores(np64(x), np64(A), np64(B), m)
+    assert_close(c.cpu().numpy(), want, 1e-3 * want.max(), "top-m ltp scores")
+
+
 def _layer_case(name):
     from synthetic import WORKLOADS, make_hidden, make_layer_weights, salient_rows
     wl = WORKLOADS[name]
@@ -75,19 +86,20 @@ def _layer_case(name):
 # the base layer and its variants: active-row keys only, Multiply fusion, one
 # probe token, the channel-reduced LTP proxy
 @pytest.mark.parametrize("name", ["layer_small", "layer_small_kv", "layer_small_mul", "layer_small_p1",
-                                  "layer_small_dlow"])
+                                  "layer_small_dlow", "layer_small_rho"])
 def test_layer_small_matches_oracle(name):
     wl, h, W, sal, pos = _layer_case(name)
     Wd = {n: t.cuda() for n, t in W.items()}
     desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k, fuse=wl.fuse,
-                        salient_rows=sal.cuda(), salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout,
+                        salient_rows=sal.cuda(), salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m,
                         kv_active_only=wl.kv_active)
     hd = h.cuda()
     out = S.spts_layer_forward(hd, pos.cuda(), desc, Wd, outputs=True)
     S.check_device_status()
     ow = O.LayerWeights(**{n: np64(t) for n, t in W.items()})
     cfg = O.LayerConfig(Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, P=wl.P, k=wl.k, fuse=wl.fuse,
-                        salient_rows=sal.numpy(), salient_shift=wl.salient_shift, kv_active=wl.kv_active)
+                        salient_rows=sal.numpy(), salient_shift=wl.salient_shift, kv_active=wl.kv_active,
+                        ltp_top_m=wl.ltp_top_m)
     tr = {}
     O.layer_forward(np64(h), pos.numpy(), ow, cfg, tr)
     s = out["s"].cpu().numpy()
@@ -110,7 +122,8 @@ def test_layer_small_matches_oracle(name):
     # within the per-call bound, then the fused score and the FFN set exactly
     # (the same fp32 operations on the same scores), then the reduced FFN
     x2 = O.bf16_round(O.rmsnorm(ha, ow.norm_ffn, cfg.eps))
-    c_want = O.ltp_scores(x2, ow.ltp_a, ow.ltp_b)
+    c_want = (O.ltp_topm_scores(x2, ow.ltp_a, ow.ltp_b, wl.ltp_top_m) if wl.ltp_top_m
+              else O.ltp_scores(x2, ow.ltp_a, ow.ltp_b))
     c = out["c"].cpu().numpy()
     assert_close(c, c_want, 1e-3 * c_want.max(), "ltp scores")
     f_want = O.fuse_scores(s.astype(np.float32), c.astype(np.float32), wl.fuse, 0.5, 0.5)

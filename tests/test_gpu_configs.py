@@ -68,7 +68,7 @@ def _run_gpu_layer(wl, h, W, pos, sal, k=None):
     Wd = {n: t.cuda() for n, t in W.items()}
     sal_d = sal.cuda() if len(sal) else None
     desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k if k is None else k, fuse=wl.fuse,
-                        salient_rows=sal_d, salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout,
+                        salient_rows=sal_d, salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m,
                         kv_active_only=wl.kv_active)
     hd = h.cuda()
     out = S.spts_layer_forward(hd, pos.cuda(), desc, Wd, outputs=True)
@@ -135,7 +135,8 @@ def _check_layer_sampled(wl, h, W, pos, sal, g, k, n_rows=40):
                                    idf[rng.choice(len(idf), n_rows // 2, replace=False)], np.arange(N - P, N)]))
     h1 = oracle_h1(rr)
     x2 = O.bf16_round(O.rmsnorm(h1, None, 1e-5))
-    c = O.ltp_scores(x2, Wn["ltp_a"], Wn["ltp_b"])
+    c = (O.ltp_topm_scores(x2, Wn["ltp_a"], Wn["ltp_b"], wl.ltp_top_m) if wl.ltp_top_m
+         else O.ltp_scores(x2, Wn["ltp_a"], Wn["ltp_b"]))
     gc = g["c"].numpy()
     assert_close(gc[rr], c, 1e-3 * c.max(), "ltp scores (sampled rows)")
     _check_topk_valid(idf, g["f"].numpy(), k, P)
@@ -154,7 +155,7 @@ def _check_layer_sampled(wl, h, W, pos, sal, g, k, n_rows=40):
 
 
 @pytest.mark.parametrize("name", ["attn_8k", "layer_32k", "layer_128k", "layer_32k_kv", "layer_128k_kv",
-                                  "layer_32k_mul", "layer_32k_dlow"])
+                                  "layer_32k_mul", "layer_32k_dlow", "layer_32k_rho"])
 def test_layer_full_size_sampled(name):
     wl = WORKLOADS[name]
     h = make_hidden(wl)

@@ -128,6 +128,24 @@ def test_ltp_identity_proxy_is_leading_norm():
     np.testing.assert_allclose(O.ltp_scores(x, A, B), np.linalg.norm(x[:, :r], axis=1), rtol=1e-15)
 
 
+
+def test_ltp_topm_brute_force_and_limits():
+    # the sum of the m largest |y| equals the best m-subset sum (brute force),
+    # the L1 norm at m = D_low and the largest |y| at m = 1
+    import itertools
+    x = O.bf16_round(rng.standard_normal((5, 16)))
+    A = O.bf16_round(rng.standard_normal((4, 16)) * 0.3)
+    B = O.bf16_round(rng.standard_normal((7, 4)) * 0.3)
+    y = O.bf16_round(x @ A.T) @ B.T
+    for m in (1, 3, 7):
+        got = O.ltp_topm_scores(x, A, B, m)
+        want = [max(sum(abs(row[j]) for j in sub) for sub in itertools.combinations(range(7), m)) for row in y]
+        np.testing.assert_allclose(got, want, rtol=1e-14)
+    np.testing.assert_allclose(O.ltp_topm_scores(x, A, B, 7), np.abs(y).sum(axis=1), rtol=1e-14)
+    np.testing.assert_allclose(O.ltp_topm_scores(x, A, B, 1), np.abs(y).max(axis=1), rtol=1e-14)
+    with pytest.raises(ValueError):
+        O.ltp_topm_scores(x, A, B, 8)
+
 def test_ltp_matches_torch_on_exact_intermediates():
     # integer inputs keep x A^T exact in bf16, so the rounding is a no-op
     D, r, Dout = 24, 6, 40

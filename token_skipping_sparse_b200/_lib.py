@@ -27,6 +27,7 @@ EXPORTS = (
     "spts_version", "spts_last_error", "spts_check_device_status", "spts_debug_set_wait_limit_ns",
     "spts_debug_get_wait_limit_ns", "spts_launch_count",
     "spts_probe_scores", "spts_probe_scores_workspace", "spts_ltp_scores", "spts_ltp_scores_workspace",
+    "spts_ltp_topm_scores", "spts_ltp_topm_scores_workspace",
     "spts_select_topk", "spts_select_topk_workspace", "spts_reduced_attention",
     "spts_reduced_attention_workspace", "spts_reduced_ffn", "spts_reduced_ffn_workspace", "spts_stage_prune",
     "spts_stage_prune_workspace", "spts_stage_prune_noalloc", "spts_rmsnorm_rows", "spts_rope", "spts_gather_rows", "spts_linear",
@@ -62,7 +63,7 @@ class LayerDesc(C.Structure):
                 ("r", C.c_int), ("P", C.c_int), ("k", C.c_int64), ("fuse", C.c_int), ("w_a", C.c_float),
                 ("w_b", C.c_float), ("eps", C.c_float), ("theta", C.c_double), ("salient_rows", C.c_void_p),
                 ("n_salient", C.c_int64), ("salient_shift", C.c_float), ("ltp_dout", C.c_int),
-                ("kv_active_only", C.c_int)]
+                ("kv_active_only", C.c_int), ("ltp_top_m", C.c_int)]
 
 
 class LayerWeights(C.Structure):
@@ -99,6 +100,8 @@ _sig("spts_probe_scores", i32, [AD, vp, vp, i32, vp, vp, i64, vp, vp, vp, sz, vp
 _sig("spts_probe_scores_workspace", sz, [AD, i32, i64])
 _sig("spts_ltp_scores", i32, [i32, vp, i64, i32, vp, i32, vp, i32, vp, vp, sz, vp])
 _sig("spts_ltp_scores_workspace", sz, [i64, i32, i32, i32])
+_sig("spts_ltp_topm_scores", i32, [i32, vp, i64, i32, vp, i32, vp, i32, i32, vp, vp, sz, vp])
+_sig("spts_ltp_topm_scores_workspace", sz, [i64, i32, i32, i32])
 _sig("spts_select_topk", i32, [vp, vp, i32, f32, f32, i64, i64, i64, vp, vp, vp, vp, sz, vp])
 _sig("spts_select_topk_workspace", sz, [i64])
 _sig("spts_reduced_attention", i32, [AD, vp, vp, i64, vp, vp, vp, i64, vp, vp, sz, vp])
@@ -214,6 +217,18 @@ def spts_ltp_scores(x, A, B, ws=None):
     return c
 
 
+def spts_ltp_topm_scores(x, A, B, top_m, ws=None):
+    """Sum of the top_m largest |y| per row of y = (x A^T) B^T (top-rho saliency)."""
+    Nc, D = x.shape
+    r, Dout = A.shape[0], B.shape[0]
+    c = torch.empty(Nc, dtype=torch.float32, device=x.device)
+    n = lib.spts_ltp_topm_scores_workspace(Nc, D, r, Dout)
+    ws = workspace(n) if ws is None else ws
+    check(lib.spts_ltp_topm_scores(BF16, ptr(x), Nc, D, ptr(A), r, ptr(B), Dout, int(top_m), ptr(c), ptr(ws),
+                                   ws.numel(), stream_ptr()))
+    return c
+
+
 def spts_select_topk(s_a, k, force_tail, s_b=None, mode=FUSE_NONE, w_a=0.5, w_b=0.5, fused=False, kth=False,
                      ws=None):
     Nc = s_a.shape[0]
@@ -326,11 +341,11 @@ def spts_inject_salience(k, q_probe, rows, shift):
 
 # ---------------------------------------------------------------- the composed layer
 def layer_desc(D, Hq, Hkv, d, F, r, P, k, fuse=FUSE_MAXNORM_ADD, w_a=0.5, w_b=0.5, eps=1e-5, theta=500000.0,
-               salient_rows=None, salient_shift=0.0, ltp_dout=0, kv_active_only=False):
+               salient_rows=None, salient_shift=0.0, ltp_dout=0, kv_active_only=False, ltp_top_m=0):
     n_sal = 0 if salient_rows is None else int(salient_rows.numel())
     desc = LayerDesc(D, Hq, Hkv, d, F, r, P, k, fuse, w_a, w_b, eps, theta,
                      None if n_sal == 0 else salient_rows.data_ptr(), n_sal, salient_shift, ltp_dout,
-                     1 if kv_active_only else 0)
+                     1 if kv_active_only else 0, int(ltp_top_m))
     desc._keep = salient_rows  # the descriptor holds a raw pointer: keep the tensor alive with it
     return desc
 

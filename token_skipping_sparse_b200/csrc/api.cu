@@ -94,6 +94,28 @@ spts_status spts_ltp_scores(spts_dtype dt, const void *x, int64_t Nc, int D, con
   return launch_ltp_bf16(x, Nc, D, A, r, B, Dout, scores, static_cast<uint32_t *>(ws), cs(stream));
 }
 
+size_t spts_ltp_topm_scores_workspace(int64_t, int, int, int) { return kStatusBytes; }
+
+spts_status spts_ltp_topm_scores(spts_dtype dt, const void *x, int64_t Nc, int D, const void *A, int r,
+                                 const void *B, int Dout, int top_m, float *scores, void *ws, size_t ws_bytes,
+                                 spts_stream stream) {
+  const char *who = "spts_ltp_topm_scores";
+  SPTS_REQUIRE(dt == SPTS_BF16, SPTS_ERR_UNSUPPORTED, "%s: only bf16 is supported", who);
+  SPTS_REQUIRE(Nc == 0 || (x && scores), SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(A && B, SPTS_ERR_INVALID, "%s: NULL weights", who);
+  SPTS_REQUIRE(Nc >= 0 && D > 0 && D % 64 == 0 && r >= 64 && r <= 256 && r % 64 == 0 &&
+                   (Dout == 256 || Dout == 512) && top_m >= 1 && top_m <= Dout,
+               SPTS_ERR_SHAPE,
+               "%s: need D%%64==0, r in {64..256} step 64, Dout in {256, 512}, 1 <= top_m <= Dout (D=%d r=%d "
+               "Dout=%d top_m=%d)",
+               who, D, r, Dout, top_m);
+  SPTS_REQUIRE(aligned(x, 16) && aligned(A, 16) && aligned(B, 16) && aligned(scores, 4), SPTS_ERR_INVALID,
+               "%s: misaligned pointer", who);
+  SPTS_TRY(check_ws(ws, ws_bytes, spts_ltp_topm_scores_workspace(Nc, D, r, Dout), who));
+  if (Nc == 0) return SPTS_OK;
+  return launch_ltp_bf16(x, Nc, D, A, r, B, Dout, scores, static_cast<uint32_t *>(ws), cs(stream), top_m);
+}
+
 // ------------------------------------------------------------------ select
 size_t spts_select_topk_workspace(int64_t Nc) {
   return kStatusBytes + Carver::round(topk_scratch_bytes(Nc));

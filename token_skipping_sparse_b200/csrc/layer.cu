@@ -88,6 +88,9 @@ spts_status check_layer(const spts_layer_desc *L, const spts_layer_weights *W, i
                  who);
     SPTS_REQUIRE(L->ltp_dout == 0 || (L->ltp_dout > 0 && L->ltp_dout % 256 == 0), SPTS_ERR_SHAPE,
                  "%s: ltp_dout must be 0 (= D) or a multiple of 256", who);
+    const int dlow = L->ltp_dout > 0 ? L->ltp_dout : L->D;
+    SPTS_REQUIRE(L->ltp_top_m == 0 || ((dlow == 256 || dlow == 512) && L->ltp_top_m >= 1 && L->ltp_top_m <= dlow),
+                 SPTS_ERR_SHAPE, "%s: ltp_top_m needs D_low in {256, 512} and 1 <= ltp_top_m <= D_low", who);
   }
   SPTS_REQUIRE(L->kv_active_only == 0 || L->kv_active_only == 1, SPTS_ERR_INVALID, "%s: kv_active_only is 0 or 1",
                who);
@@ -223,7 +226,8 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   int32_t *idx_f = o.idx_ffn ? o.idx_ffn : b.idx_f;
   SPTS_TRY(launch_rmsnorm_rows(h, nullptr, Nc, D, W->norm_ffn, L->eps, b.xn, s));
   SPTS_TRY(mark(11));
-  SPTS_TRY(launch_ltp_bf16(b.xn, Nc, D, W->ltp_a, L->r, W->ltp_b, L->ltp_dout > 0 ? L->ltp_dout : D, c, st, s));
+  SPTS_TRY(launch_ltp_bf16(b.xn, Nc, D, W->ltp_a, L->r, W->ltp_b, L->ltp_dout > 0 ? L->ltp_dout : D, c, st, s,
+                           L->ltp_top_m));
   SPTS_TRY(mark(12));
   SPTS_TRY(launch_select_topk(sc, c, L->fuse, L->w_a, L->w_b, Nc, k, P, idx_f, f, nullptr, st, b.topk, s));
   SPTS_TRY(launch_gather_rows(b.xn, Nc, idx_f, k, static_cast<int64_t>(D) * 2, b.xsel, nullptr, nullptr, st, s));

@@ -9,6 +9,11 @@
 //   phase 2  Y = T B^T   (M=128, N=256 per chunk, K=r), chunk by chunk over
 //            the Dout outputs into two ping-pong TMEM accumulators; the
 //            epilogue warps fold every chunk into a per-row sum of squares.
+// With top_m > 0 (D_low = Dout <= 512, both chunks resident in TMEM) the
+// score is instead the sum of the top_m largest |y| of the row (top-rho
+// channel saliency, Table E): each row's thread finds its top_m-th largest
+// |y| by a bitwise search over the float bits (31 counting passes over the
+// row in TMEM), then sums the values above it plus the ties it needs.
 // Per row only 2*D bytes of X are read from HBM; A and B (2 x r x D bf16)
 // are shared by all CTAs through L2.  Waits are bounded.
 #include "host.hpp"
@@ -29,6 +34,7 @@ constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 256;
 
 struct Params {
   int M, D, r, Dout;
+  int top_m;  // 0: L2 norm of y; > 0: sum of the top_m largest |y| (Dout <= 512)
   float *scores;
   uint32_t *status;
   uint64_t wait_ns;
@@ -180,7 +186,52 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(ts_ready);
     }
     float ss = 0.f;
-    for (int nc = 0; ok && nc < nch; ++nc) {
+    if (p.top_m > 0) {
+      // both chunks (Dout <= 512 columns) resident: acc 0 = columns [0, 256)
+      for (int nc = 0; ok && nc < nch; ++nc) {
+        const bool okw = mbar_wait(&acc_full[nc], 0, abort_flag, p.status, p.wait_ns, 0x58u);
+        ok = __all_sync(0xffffffffu, okw);
+      }
+      if (ok) {
+        tc_fence_after();
+        // largest T with at least top_m values of |y| >= T (|y| bits order as uints)
+        uint32_t T = 0u;
+#pragma unroll 1
+        for (int b = 30; b >= 0; --b) {
+          const uint32_t cand = T | (1u << b);
+          int cnt = 0;
+#pragma unroll 1
+          for (int c0 = 0; c0 < p.Dout; c0 += 32) {
+            uint32_t y[32];
+            tmem_ld32(lane_base + c0, y);
+            tmem_ld_wait();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) cnt += (y[t] & 0x7FFFFFFFu) >= cand;
+          }
+          if (cnt >= p.top_m) T = cand;
+        }
+        int gt = 0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < p.Dout; c0 += 32) {
+          uint32_t y[32];
+          tmem_ld32(lane_base + c0, y);
+          tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const uint32_t u = y[t] & 0x7FFFFFFFu;
+            if (u > T) {
+              ss += __uint_as_float(u);
+              ++gt;
+            }
+          }
+        }
+        ss += static_cast<float>(p.top_m - gt) * __uint_as_float(T);  // the ties at the threshold
+        tc_fence_before();
+        for (int nc = 0; nc < nch; ++nc) mbar_arrive(&acc_empty[nc]);
+      }
+      if (ok && m0 + rr < p.M) p.scores[m0 + rr] = ss;
+    }
+    for (int nc = 0; ok && p.top_m == 0 && nc < nch; ++nc) {
       const int acc = nc & 1;
       const bool okw = mbar_wait(&acc_full[acc], (nc >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x57u);
       if (!__all_sync(0xffffffffu, okw)) {
@@ -202,7 +253,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }
-    if (ok && m0 + rr < p.M) p.scores[m0 + rr] = sqrtf(ss);
+    if (ok && p.top_m == 0 && m0 + rr < p.M) p.scores[m0 + rr] = sqrtf(ss);
   }
   __syncthreads();
   if (warp == 1) {
@@ -214,13 +265,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 }  // namespace
 
 spts_status launch_ltp_bf16(const void *x, int64_t Nc, int D, const void *A, int r, const void *B, int Dout,
-                            float *scores, uint32_t *status, cudaStream_t s) {
+                            float *scores, uint32_t *status, cudaStream_t s, int top_m) {
   if (Nc == 0) return SPTS_OK;
   CUtensorMap tx, ta, tb;
   SPTS_TRY(tmap_bf16_2d(&tx, x, static_cast<uint64_t>(Nc), D, D, 128));
   SPTS_TRY(tmap_bf16_2d(&ta, A, r, D, D, static_cast<uint32_t>(r)));
   SPTS_TRY(tmap_bf16_2d(&tb, B, Dout, r, r, 256));
-  Params p{static_cast<int>(Nc), D, r, Dout, scores, status, wait_limit_ns()};
+  Params p{static_cast<int>(Nc), D, r, Dout, top_m, scores, status, wait_limit_ns()};
   SPTS_CUDA_TRY(
       cudaFuncSetAttribute(ltp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM_BYTES)));
   ltp_kernel<<<static_cast<unsigned>((Nc + 127) / 128), THREADS, SMEM_BYTES, s>>>(tx, ta, tb, p);

@@ -66,8 +66,9 @@ spts_status launch_probe_bf16(const void *q, const int32_t *qpos, int P, const v
                               uint32_t *status, cudaStream_t s);
 size_t probe_bf16_stats_bytes(int P, int Hq, int64_t Nc);
 
+// top_m > 0 (Dout <= 512): score = sum of the top_m largest |y| instead of ||y||_2.
 spts_status launch_ltp_bf16(const void *x, int64_t Nc, int D, const void *A, int r, const void *B, int Dout,
-                            float *scores, uint32_t *status, cudaStream_t s);
+                            float *scores, uint32_t *status, cudaStream_t s, int top_m = 0);
 
 spts_status launch_attention_bf16(const void *q, const int32_t *qpos, int64_t m, const void *k, const void *v,
                                   const int32_t *kpos, int64_t Nc, int Hq, int Hkv, float scale, void *o,
