@@ -167,7 +167,7 @@ class LayerCase:
         wl = self.wl
         return self.S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k if k is None else k,
                                  fuse=wl.fuse, salient_rows=self.sal if len(self.sal) else None,
-                                 salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m,
+                                 salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m, seq_pool=0,
                                  kv_active_only=wl.kv_active)
 
 

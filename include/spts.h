@@ -72,8 +72,18 @@ typedef enum { SPTS_F32 = 0, SPTS_BF16 = 1 } spts_dtype;
 
 /* Score fusion of Table D: f = s (NONE); f = w_a*s/max(s) + w_b*c/max(c)
  * (MAXNORM_ADD, each max over all Nc entries, a term with max 0 adds 0);
- * f = s*c (MULTIPLY, the criterion C*S of Table 6). */
-typedef enum { SPTS_FUSE_NONE = 0, SPTS_FUSE_MAXNORM_ADD = 1, SPTS_FUSE_MULTIPLY = 2 } spts_fuse;
+ * f = s*c (MULTIPLY, the criterion C*S of Table 6);
+ * f = w_a*(s - mean s)/std s + w_b*(c - mean c)/std c (STD_ADD: population
+ * mean and standard deviation over all Nc entries, computed in fp64 and
+ * rounded to fp32; a term with std 0 adds 0).  All in fp32 with one rounding
+ * per operation.  Sequential Select is spts_select_sequential. */
+typedef enum {
+  SPTS_FUSE_NONE = 0,
+  SPTS_FUSE_MAXNORM_ADD = 1,
+  SPTS_FUSE_MULTIPLY = 2,
+  SPTS_FUSE_STD_ADD = 3,
+  SPTS_FUSE_SEQUENTIAL = 4 /* layer descriptor only: see spts_layer_desc.seq_pool */
+} spts_fuse;
 
 /* Attention geometry.  scale <= 0 means 1/sqrt(d).
  * Supported: F32 with d in {64, 128}; BF16 with d = 128 and Hq/Hkv in {1,2,4,8}. */
@@ -276,6 +286,16 @@ SPTS_API size_t spts_linear_workspace(void);
 SPTS_API spts_status spts_inject_salience(void *k, int64_t Nc, const void *q_probe, int P, int Hq, int Hkv, int d,
                                  const int32_t *rows, int64_t n_rows, float shift, spts_stream stream);
 
+/* Sequential Select of Table D (reading: the pages name it only): the pool
+ * = the top-k_pool candidates by s_a (the last force_tail always kept, ties
+ * to the lower index), then the top-k of the pool by s_b under the same
+ * rules; idx_out [k] holds candidate indices, ascending.
+ * Limits: 0 <= force_tail <= k <= k_pool <= Nc < 2^31. */
+SPTS_API spts_status spts_select_sequential(const float *s_a, const float *s_b, int64_t Nc, int64_t k_pool,
+                                            int64_t k, int64_t force_tail, int32_t *idx_out, void *ws,
+                                            size_t ws_bytes, spts_stream stream);
+SPTS_API size_t spts_select_sequential_workspace(int64_t Nc);
+
 /* ---------------------------------------------------------------------- */
 /* The composed layer (probe -> reduced MHA -> LTP -> reduced FFN)         */
 /* ---------------------------------------------------------------------- */
@@ -302,6 +322,10 @@ typedef struct {
   /* > 0: the LTP score is the top-rho channel saliency, the sum of the
    * ltp_top_m largest |y| (needs ltp_dout in {256, 512}); 0: ||y||_2.      */
   int ltp_top_m;
+  /* fuse == SPTS_FUSE_SEQUENTIAL: the pool of the FFN selection (top
+   * seq_pool rows by the probe score, then the top k of them by the LTP
+   * score); 0 means min(Nc, 2k).  The layer's fused output f is then c.   */
+  int64_t seq_pool;
 } spts_layer_desc;
 
 typedef struct {

@@ -42,12 +42,15 @@ __all__ = [
     "bf16_round", "rmsnorm", "rope", "probe_scores", "ltp_scores", "ltp_topm_scores", "fuse_scores",
     "select_topk", "reduced_attention", "attention_residual", "reduced_ffn",
     "stage_prune", "inject_salience", "LayerWeights", "LayerConfig", "layer_forward",
-    "msdp_forward", "MsdpConfig", "FUSE_NONE", "FUSE_MAXNORM_ADD", "FUSE_MULTIPLY",
+    "msdp_forward", "MsdpConfig", "FUSE_NONE", "FUSE_MAXNORM_ADD", "FUSE_MULTIPLY", "FUSE_STD_ADD",
+    "FUSE_SEQUENTIAL", "select_sequential",
 ]
 
 FUSE_NONE = 0
 FUSE_MAXNORM_ADD = 1
 FUSE_MULTIPLY = 2
+FUSE_STD_ADD = 3
+FUSE_SEQUENTIAL = 4    # layer setting: select_sequential
 
 
 # --------------------------------------------------------------------------
@@ -187,6 +190,10 @@ def fuse_scores(s, c, mode, w_a=0.5, w_b=0.5):
       MULTIPLY:    f = s * c
       MAXNORM_ADD: f = w_a * (s / max s) + w_b * (c / max c), each max over
                    all candidates; a term whose max is 0 contributes 0.
+      STD_ADD:     f = w_a * ((s - mean s) / std s) + w_b * ((c - mean c) / std c)
+                   (reading of the name "Std-Add"): population mean and
+                   standard deviation over all candidates, exact in fp64 and
+                   rounded to fp32; a term whose std is 0 contributes 0.
     Each operation rounds to fp32 (no fused multiply-add), in this order.
     """
     s = np.asarray(s, dtype=np.float32)
@@ -201,6 +208,16 @@ def fuse_scores(s, c, mode, w_a=0.5, w_b=0.5):
         ta = (np.float32(w_a) * (s / ms)).astype(np.float32) if ms > 0 else np.zeros_like(s)
         tb = (np.float32(w_b) * (c / mc)).astype(np.float32) if mc > 0 else np.zeros_like(c)
         return (ta + tb).astype(np.float32)
+    if mode == FUSE_STD_ADD:
+        def standardised(x, w):
+            x64 = x.astype(np.float64)
+            mu = math.fsum(x64) / len(x64)
+            sd = math.sqrt(math.fsum((x64 - mu) ** 2) / len(x64))
+            mu32, sd32 = np.float32(mu), np.float32(sd)
+            if not sd32 > 0:
+                return np.zeros_like(x)
+            return (np.float32(w) * ((x - mu32).astype(np.float32) / sd32).astype(np.float32)).astype(np.float32)
+        return (standardised(s, w_a) + standardised(c, w_b)).astype(np.float32)
     raise ValueError(f"unknown fusion mode {mode}")
 
 
@@ -230,6 +247,20 @@ def select_topk(f, k, force_tail):
     idx = np.concatenate([chosen, np.arange(n_free, Nc)]).astype(np.int64)
     tau = float(f[order[k_free - 1]]) if k_free > 0 else float("nan")
     return idx, tau
+
+
+def select_sequential(s, c, k_pool, k, force_tail):
+    """Sequential Select of Table D (reading: the pages only name it).
+
+    The attention-based score narrows the candidates first and the
+    transformation score decides second: the pool is select_topk(s, k_pool),
+    then the k of the pool with the largest c under the same rules (the
+    forced tail stays, ties go to the lower index).  Returns (indices
+    ascending, threshold of the second selection).
+    """
+    pool, _ = select_topk(np.asarray(s, dtype=np.float32), k_pool, force_tail)
+    local, tau = select_topk(np.asarray(c, dtype=np.float32)[pool], k, force_tail)
+    return pool[local], tau
 
 
 # --------------------------------------------------------------------------
@@ -343,6 +374,7 @@ class LayerConfig:
     salient_shift: float = 0.0
     kv_active: bool = False    # reduced attention over the active rows' keys only
     ltp_top_m: int = 0         # > 0: LTP saliency = sum of the top m |y| (Table E); 0: L2 norm
+    seq_pool: int = 0          # FUSE_SEQUENTIAL: pool size (0: min(Nc, 2k))
 
 
 def inject_salience(kk, q_probe, rows, shift, Hkv):
@@ -400,8 +432,13 @@ def layer_forward(h, pos, W: LayerWeights, cfg: LayerConfig, trace: dict | None 
     x_ffn = bf16_round(rmsnorm(h1, W.norm_ffn, cfg.eps))
     c = (ltp_topm_scores(x_ffn, W.ltp_a, W.ltp_b, cfg.ltp_top_m) if cfg.ltp_top_m > 0
          else ltp_scores(x_ffn, W.ltp_a, W.ltp_b))
-    f = fuse_scores(s32, c.astype(np.float32), cfg.fuse, cfg.w_a, cfg.w_b)
-    idx_f, tau_f = select_topk(f, k, P)
+    if cfg.fuse == FUSE_SEQUENTIAL:
+        pool = cfg.seq_pool if cfg.seq_pool > 0 else min(Nc, 2 * k)
+        f = c.astype(np.float32)
+        idx_f, tau_f = select_sequential(s32, f, pool, k, P)
+    else:
+        f = fuse_scores(s32, c.astype(np.float32), cfg.fuse, cfg.w_a, cfg.w_b)
+        idx_f, tau_f = select_topk(f, k, P)
     h2 = reduced_ffn(h1, idx_f, W.norm_ffn, cfg.eps, W.w_gate, W.w_up, W.w_down)
     t.update(x_ffn=x_ffn, c=c, f=f, idx_ffn=idx_f, tau_ffn=tau_f, h_out=h2)
     return h2, f

@@ -21,9 +21,10 @@ from fractions import Fraction
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "keep_rows", "salient_rows", "make_qkv_f32",
-           "make_hidden", "make_layer_weights", "FUSE_NONE", "FUSE_MAXNORM_ADD", "FUSE_MULTIPLY"]
+           "make_hidden", "make_layer_weights", "FUSE_NONE", "FUSE_MAXNORM_ADD", "FUSE_MULTIPLY",
+           "FUSE_STD_ADD", "FUSE_SEQUENTIAL"]
 
-FUSE_NONE, FUSE_MAXNORM_ADD, FUSE_MULTIPLY = 0, 1, 2
+FUSE_NONE, FUSE_MAXNORM_ADD, FUSE_MULTIPLY, FUSE_STD_ADD, FUSE_SEQUENTIAL = 0, 1, 2, 3, 4
 
 
 @dataclass(frozen=True)
@@ -86,7 +87,8 @@ WORKLOADS = {
 #   _mul   the Multiply fusion f = s * c for the FFN selection;
 #   _p1    a single probe token;
 #   _dlow  the channel-reduced LTP proxy, D_low = 512 output channels, r = 192;
-#   _rho   that proxy with top-rho saliency, rho = 0.2: the top 103 of 512 |y|.
+#   _rho   that proxy with top-rho saliency, rho = 0.2: the top 103 of 512 |y|;
+#   _std   the Std-Add fusion; _seq the Sequential Select (pool 2k).
 for _base in ("layer_32k", "layer_128k", "layer_small"):
     _w = WORKLOADS[_base]
     WORKLOADS[_base + "_kv"] = replace(_w, name=_base + "_kv", kv_active=True)
@@ -94,6 +96,8 @@ for _base in ("layer_32k", "layer_128k", "layer_small"):
     WORKLOADS[_base + "_p1"] = replace(_w, name=_base + "_p1", P=1)
     WORKLOADS[_base + "_dlow"] = replace(_w, name=_base + "_dlow", ltp_dout=512, r=192)
     WORKLOADS[_base + "_rho"] = replace(_w, name=_base + "_rho", ltp_dout=512, r=192, ltp_top_m=103)
+    WORKLOADS[_base + "_std"] = replace(_w, name=_base + "_std", fuse=FUSE_STD_ADD)
+    WORKLOADS[_base + "_seq"] = replace(_w, name=_base + "_seq", fuse=FUSE_SEQUENTIAL)
 del _base, _w
 
 

@@ -86,12 +86,12 @@ def _layer_case(name):
 # the base layer and its variants: active-row keys only, Multiply fusion, one
 # probe token, the channel-reduced LTP proxy
 @pytest.mark.parametrize("name", ["layer_small", "layer_small_kv", "layer_small_mul", "layer_small_p1",
-                                  "layer_small_dlow", "layer_small_rho"])
+                                  "layer_small_dlow", "layer_small_rho", "layer_small_std", "layer_small_seq"])
 def test_layer_small_matches_oracle(name):
     wl, h, W, sal, pos = _layer_case(name)
     Wd = {n: t.cuda() for n, t in W.items()}
     desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k, fuse=wl.fuse,
-                        salient_rows=sal.cuda(), salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m,
+                        salient_rows=sal.cuda(), salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m, seq_pool=0,
                         kv_active_only=wl.kv_active)
     hd = h.cuda()
     out = S.spts_layer_forward(hd, pos.cuda(), desc, Wd, outputs=True)
@@ -126,10 +126,15 @@ def test_layer_small_matches_oracle(name):
               else O.ltp_scores(x2, ow.ltp_a, ow.ltp_b))
     c = out["c"].cpu().numpy()
     assert_close(c, c_want, 1e-3 * c_want.max(), "ltp scores")
-    f_want = O.fuse_scores(s.astype(np.float32), c.astype(np.float32), wl.fuse, 0.5, 0.5)
-    assert np.array_equal(out["f"].cpu().numpy().view(np.uint32), f_want.view(np.uint32)), "fused score"
     idf = out["idx_ffn"].cpu().numpy()
-    assert np.array_equal(idf, O.select_topk(f_want, wl.k, wl.P)[0]), "FFN selection"
+    if wl.fuse == O.FUSE_SEQUENTIAL:  # the pool by s, then the k by c; f is c
+        assert np.array_equal(out["f"].cpu().numpy(), c)
+        want_f = O.select_sequential(s.astype(np.float32), c.astype(np.float32), min(wl.N, 2 * wl.k), wl.k, wl.P)[0]
+        assert np.array_equal(idf, want_f), "FFN selection"
+    else:
+        f_want = O.fuse_scores(s.astype(np.float32), c.astype(np.float32), wl.fuse, 0.5, 0.5)
+        assert np.array_equal(out["f"].cpu().numpy().view(np.uint32), f_want.view(np.uint32)), "fused score"
+        assert np.array_equal(idf, O.select_topk(f_want, wl.k, wl.P)[0]), "FFN selection"
     h_want = O.reduced_ffn(ha, idf, ow.norm_ffn, cfg.eps, ow.w_gate, ow.w_up, ow.w_down)
     assert_close(np64(hd), h_want, 2e-2, "h out (reduced FFN on the GPU's h')")
     # the composed layer against the oracle's own chain: two bf16-stored stages

@@ -68,7 +68,7 @@ def _run_gpu_layer(wl, h, W, pos, sal, k=None):
     Wd = {n: t.cuda() for n, t in W.items()}
     sal_d = sal.cuda() if len(sal) else None
     desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k if k is None else k, fuse=wl.fuse,
-                        salient_rows=sal_d, salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m,
+                        salient_rows=sal_d, salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m, seq_pool=0,
                         kv_active_only=wl.kv_active)
     hd = h.cuda()
     out = S.spts_layer_forward(hd, pos.cuda(), desc, Wd, outputs=True)
@@ -139,7 +139,11 @@ def _check_layer_sampled(wl, h, W, pos, sal, g, k, n_rows=40):
          else O.ltp_scores(x2, Wn["ltp_a"], Wn["ltp_b"]))
     gc = g["c"].numpy()
     assert_close(gc[rr], c, 1e-3 * c.max(), "ltp scores (sampled rows)")
-    _check_topk_valid(idf, g["f"].numpy(), k, P)
+    if wl.fuse == O.FUSE_SEQUENTIAL:  # the pool by s, then the k by c (the kernel's own scores)
+        want_f = O.select_sequential(gs, gc, min(N, 2 * k), k, P)[0]
+        assert np.array_equal(idf, want_f), "sequential FFN selection"
+    else:
+        _check_topk_valid(idf, g["f"].numpy(), k, P)
 
     # reduced FFN on sampled rows: selected rows get the FFN delta, others stay
     ho = g["h_out"].numpy()
@@ -155,7 +159,8 @@ def _check_layer_sampled(wl, h, W, pos, sal, g, k, n_rows=40):
 
 
 @pytest.mark.parametrize("name", ["attn_8k", "layer_32k", "layer_128k", "layer_32k_kv", "layer_128k_kv",
-                                  "layer_32k_mul", "layer_32k_dlow", "layer_32k_rho"])
+                                  "layer_32k_mul", "layer_32k_dlow", "layer_32k_rho", "layer_32k_std",
+                                  "layer_32k_seq"])
 def test_layer_full_size_sampled(name):
     wl = WORKLOADS[name]
     h = make_hidden(wl)

@@ -111,7 +111,7 @@ def test_gather_rows_and_bad_index():
 # ---------------------------------------------------------------- selection
 @pytest.mark.parametrize("Nc,k,tail", [(1000, 300, 16), (1000, 1000, 16), (1000, 16, 16), (60000, 12000, 128),
                                        (131072, 26214, 128), (7, 3, 0), (1, 1, 1)])
-@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
 def test_select_topk_bit_exact(Nc, k, tail, mode):
     s = rng.random(Nc).astype(np.float32)
     c = (rng.random(Nc) * 30).astype(np.float32)
@@ -129,6 +129,17 @@ def test_select_topk_bit_exact(Nc, k, tail, mode):
     else:
         assert np.isnan(kth.item())
 
+
+
+@pytest.mark.parametrize("Nc,k_pool,k,tail", [(1000, 600, 300, 16), (60000, 24000, 12000, 128),
+                                              (131072, 52428, 26214, 128), (500, 500, 100, 0), (300, 40, 40, 8)])
+def test_select_sequential_matches_oracle(Nc, k_pool, k, tail):
+    s = rng.random(Nc).astype(np.float32)
+    c = (rng.random(Nc) * 30).astype(np.float32)
+    c[rng.integers(0, Nc, Nc // 10)] = 7.0         # ties in the second criterion
+    idx = S.spts_select_sequential(torch.from_numpy(s).cuda(), torch.from_numpy(c).cuda(), k_pool, k, tail)
+    want, _ = O.select_sequential(s, c, k_pool, k, tail)
+    assert np.array_equal(idx.cpu().numpy(), want)
 
 def test_select_rejects_bad_sizes():
     s = torch.rand(10).cuda()

@@ -202,6 +202,44 @@ def test_select_topk_brute_force_with_ties(n, k, tail):
             assert tau == min(f[i] for i in idx[: k - tail])
 
 
+
+def test_fuse_std_add_is_weighted_zscores():
+    # Std-Add reduces to the library z-score (population std) of each score
+    from scipy.stats import zscore
+    s = rng.random(500).astype(np.float32)
+    c = (rng.random(500) * 30).astype(np.float32)
+    f = O.fuse_scores(s, c, O.FUSE_STD_ADD, 0.25, 0.75)
+    want = 0.25 * zscore(s.astype(np.float64)) + 0.75 * zscore(c.astype(np.float64))
+    np.testing.assert_allclose(f, want, rtol=0, atol=2e-6)
+    # a constant score has std 0 and contributes nothing
+    f0 = O.fuse_scores(np.full(500, 0.3, np.float32), c, O.FUSE_STD_ADD, 0.5, 0.5)
+    np.testing.assert_allclose(f0, 0.5 * zscore(c.astype(np.float64)), rtol=0, atol=2e-6)
+
+
+@pytest.mark.parametrize("k_pool", [20, 33, 60])
+def test_select_sequential_reductions(k_pool):
+    # pool of everything: the selection by c alone; pool of size k: the
+    # selection by s alone; otherwise a subset of the pool holding the tail
+    n, k, tail = 60, 20, 4
+    s = rng.random(n).astype(np.float32)
+    c = rng.random(n).astype(np.float32)
+    c[rng.integers(0, n, 10)] = 0.5
+    idx, _ = O.select_sequential(s, c, k_pool, k, tail)
+    pool, _ = O.select_topk(s, k_pool, tail)
+    assert len(idx) == k and np.all(np.diff(idx) > 0)
+    assert set(idx) <= set(pool) and set(range(n - tail, n)) <= set(idx)
+    if k_pool == n:
+        assert np.array_equal(idx, O.select_topk(c, k, tail)[0])
+    if k_pool == k:
+        assert np.array_equal(idx, pool)
+    # brute force inside the pool: no dropped pool member beats a kept one
+    free_pool = [i for i in pool if i < n - tail]
+    kept = [i for i in idx if i < n - tail]
+    dropped = [i for i in free_pool if i not in kept]
+    for a in kept:
+        for b in dropped:
+            assert c[a] > c[b] or (c[a] == c[b] and a < b)
+
 def test_select_keep_all_and_errors():
     f = rng.random(33).astype(np.float32)
     idx, _ = O.select_topk(f, 33, 5)

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libspts.so")
 
 OK, ERR_INVALID, ERR_SHAPE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
 F32, BF16 = 0, 1
-FUSE_NONE, FUSE_MAXNORM_ADD, FUSE_MULTIPLY = 0, 1, 2
+FUSE_NONE, FUSE_MAXNORM_ADD, FUSE_MULTIPLY, FUSE_STD_ADD, FUSE_SEQUENTIAL = 0, 1, 2, 3, 4
 EPI_STORE, EPI_ROPE, EPI_SWIGLU, EPI_SCATTER_ADD = 0, 1, 2, 3
 
 EXPORTS = (
@@ -28,7 +28,8 @@ EXPORTS = (
     "spts_debug_get_wait_limit_ns", "spts_launch_count",
     "spts_probe_scores", "spts_probe_scores_workspace", "spts_ltp_scores", "spts_ltp_scores_workspace",
     "spts_ltp_topm_scores", "spts_ltp_topm_scores_workspace",
-    "spts_select_topk", "spts_select_topk_workspace", "spts_reduced_attention",
+    "spts_select_topk", "spts_select_topk_workspace", "spts_select_sequential", "spts_select_sequential_workspace",
+    "spts_reduced_attention",
     "spts_reduced_attention_workspace", "spts_reduced_ffn", "spts_reduced_ffn_workspace", "spts_stage_prune",
     "spts_stage_prune_workspace", "spts_stage_prune_noalloc", "spts_rmsnorm_rows", "spts_rope", "spts_gather_rows", "spts_linear",
     "spts_linear_workspace", "spts_inject_salience", "spts_layer_forward", "spts_layer_forward_workspace",
@@ -63,7 +64,7 @@ class LayerDesc(C.Structure):
                 ("r", C.c_int), ("P", C.c_int), ("k", C.c_int64), ("fuse", C.c_int), ("w_a", C.c_float),
                 ("w_b", C.c_float), ("eps", C.c_float), ("theta", C.c_double), ("salient_rows", C.c_void_p),
                 ("n_salient", C.c_int64), ("salient_shift", C.c_float), ("ltp_dout", C.c_int),
-                ("kv_active_only", C.c_int), ("ltp_top_m", C.c_int)]
+                ("kv_active_only", C.c_int), ("ltp_top_m", C.c_int), ("seq_pool", C.c_int64)]
 
 
 class LayerWeights(C.Structure):
@@ -104,6 +105,8 @@ _sig("spts_ltp_topm_scores", i32, [i32, vp, i64, i32, vp, i32, vp, i32, i32, vp,
 _sig("spts_ltp_topm_scores_workspace", sz, [i64, i32, i32, i32])
 _sig("spts_select_topk", i32, [vp, vp, i32, f32, f32, i64, i64, i64, vp, vp, vp, vp, sz, vp])
 _sig("spts_select_topk_workspace", sz, [i64])
+_sig("spts_select_sequential", i32, [vp, vp, i64, i64, i64, i64, vp, vp, sz, vp])
+_sig("spts_select_sequential_workspace", sz, [i64])
 _sig("spts_reduced_attention", i32, [AD, vp, vp, i64, vp, vp, vp, i64, vp, vp, sz, vp])
 _sig("spts_reduced_attention_workspace", sz, [AD, i64, i64])
 _sig("spts_reduced_ffn", i32, [i32, vp, i64, i32, vp, i64, vp, f32, vp, vp, vp, i32, vp, sz, vp])
@@ -229,6 +232,17 @@ def spts_ltp_topm_scores(x, A, B, top_m, ws=None):
     return c
 
 
+def spts_select_sequential(s_a, s_b, k_pool, k, force_tail, ws=None):
+    """Top-k_pool by s_a (tail forced), then the top-k of that pool by s_b; indices ascending."""
+    Nc = s_a.shape[0]
+    idx = torch.empty(k, dtype=torch.int32, device=s_a.device)
+    n = lib.spts_select_sequential_workspace(Nc)
+    ws = workspace(n) if ws is None else ws
+    check(lib.spts_select_sequential(ptr(s_a), ptr(s_b), Nc, k_pool, k, force_tail, ptr(idx), ptr(ws), ws.numel(),
+                                     stream_ptr()))
+    return idx
+
+
 def spts_select_topk(s_a, k, force_tail, s_b=None, mode=FUSE_NONE, w_a=0.5, w_b=0.5, fused=False, kth=False,
                      ws=None):
     Nc = s_a.shape[0]
@@ -341,11 +355,11 @@ def spts_inject_salience(k, q_probe, rows, shift):
 
 # ---------------------------------------------------------------- the composed layer
 def layer_desc(D, Hq, Hkv, d, F, r, P, k, fuse=FUSE_MAXNORM_ADD, w_a=0.5, w_b=0.5, eps=1e-5, theta=500000.0,
-               salient_rows=None, salient_shift=0.0, ltp_dout=0, kv_active_only=False, ltp_top_m=0):
+               salient_rows=None, salient_shift=0.0, ltp_dout=0, kv_active_only=False, ltp_top_m=0, seq_pool=0):
     n_sal = 0 if salient_rows is None else int(salient_rows.numel())
     desc = LayerDesc(D, Hq, Hkv, d, F, r, P, k, fuse, w_a, w_b, eps, theta,
                      None if n_sal == 0 else salient_rows.data_ptr(), n_sal, salient_shift, ltp_dout,
-                     1 if kv_active_only else 0, int(ltp_top_m))
+                     1 if kv_active_only else 0, int(ltp_top_m), int(seq_pool))
     desc._keep = salient_rows  # the descriptor holds a raw pointer: keep the tensor alive with it
     return desc
 

@@ -125,7 +125,8 @@ spts_status spts_select_topk(const float *s_a, const float *s_b, spts_fuse mode,
                              int64_t Nc, int64_t k, int64_t force_tail, int32_t *idx_out, float *fused_out,
                              float *kth_score_out, void *ws, size_t ws_bytes, spts_stream stream) {
   const char *who = "spts_select_topk";
-  SPTS_REQUIRE(mode == SPTS_FUSE_NONE || mode == SPTS_FUSE_MAXNORM_ADD || mode == SPTS_FUSE_MULTIPLY,
+  SPTS_REQUIRE(mode == SPTS_FUSE_NONE || mode == SPTS_FUSE_MAXNORM_ADD || mode == SPTS_FUSE_MULTIPLY ||
+                   mode == SPTS_FUSE_STD_ADD,
                SPTS_ERR_INVALID, "%s: unknown fusion mode %d", who, static_cast<int>(mode));
   SPTS_REQUIRE(Nc == 0 || (s_a && idx_out && (mode == SPTS_FUSE_NONE || s_b)), SPTS_ERR_INVALID, "%s: NULL argument", who);
   SPTS_REQUIRE(0 <= force_tail && force_tail <= k && k <= Nc && Nc < (int64_t(1) << 31), SPTS_ERR_SHAPE,
@@ -140,6 +141,28 @@ spts_status spts_select_topk(const float *s_a, const float *s_b, spts_fuse mode,
   void *scratch = cv.take(topk_scratch_bytes(Nc));
   return launch_select_topk(s_a, s_b, mode, w_a, w_b, Nc, k, force_tail, idx_out, fused_out, kth_score_out,
                             cv.status(), scratch, cs(stream));
+}
+
+size_t spts_select_sequential_workspace(int64_t Nc) {
+  return kStatusBytes + Carver::round(select_sequential_scratch_bytes(Nc));
+}
+
+spts_status spts_select_sequential(const float *s_a, const float *s_b, int64_t Nc, int64_t k_pool, int64_t k,
+                                   int64_t force_tail, int32_t *idx_out, void *ws, size_t ws_bytes,
+                                   spts_stream stream) {
+  const char *who = "spts_select_sequential";
+  SPTS_REQUIRE(Nc == 0 || (s_a && s_b && idx_out), SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(0 <= force_tail && force_tail <= k && k <= k_pool && k_pool <= Nc && Nc < (int64_t(1) << 31),
+               SPTS_ERR_SHAPE, "%s: need 0 <= force_tail <= k <= k_pool <= Nc < 2^31 (tail=%lld k=%lld pool=%lld "
+               "Nc=%lld)", who, static_cast<long long>(force_tail), static_cast<long long>(k),
+               static_cast<long long>(k_pool), static_cast<long long>(Nc));
+  SPTS_REQUIRE(aligned(s_a, 4) && aligned(s_b, 4) && aligned(idx_out, 4), SPTS_ERR_INVALID,
+               "%s: misaligned pointer", who);
+  SPTS_TRY(check_ws(ws, ws_bytes, spts_select_sequential_workspace(Nc), who));
+  if (Nc == 0 || k == 0) return SPTS_OK;
+  Carver cv(ws, ws_bytes);
+  void *scratch = cv.take(select_sequential_scratch_bytes(Nc));
+  return launch_select_sequential(s_a, s_b, Nc, k_pool, k, force_tail, idx_out, scratch, cv.status(), cs(stream));
 }
 
 // ------------------------------------------------------------------ attention

@@ -39,7 +39,7 @@ void carve(Carver &cv, const spts_layer_desc *L, int64_t Nc, LayerBufs &b) {
   b.idx_a = static_cast<int32_t *>(cv.take(k * 4));
   b.idx_f = static_cast<int32_t *>(cv.take(k * 4));
   b.qpos = static_cast<int32_t *>(cv.take(k * 4));
-  b.topk = cv.take(topk_scratch_bytes(Nc));
+  b.topk = cv.take(select_sequential_scratch_bytes(Nc));  // also covers the plain top-k
   b.ksel = cv.take(k * hk * 2);
 }
 
@@ -84,8 +84,10 @@ spts_status check_layer(const spts_layer_desc *L, const spts_layer_weights *W, i
                  "%s: need F %% 128 == 0 and r in {64,...,256} step 64", who);
     SPTS_REQUIRE(W->w_gate && W->w_up && W->w_down && W->ltp_a && W->ltp_b, SPTS_ERR_INVALID,
                  "%s: FFN / LTP weights missing", who);
-    SPTS_REQUIRE(L->fuse >= SPTS_FUSE_NONE && L->fuse <= SPTS_FUSE_MULTIPLY, SPTS_ERR_INVALID, "%s: bad fusion",
+    SPTS_REQUIRE(L->fuse >= SPTS_FUSE_NONE && L->fuse <= SPTS_FUSE_SEQUENTIAL, SPTS_ERR_INVALID, "%s: bad fusion",
                  who);
+    SPTS_REQUIRE(L->fuse != SPTS_FUSE_SEQUENTIAL || L->seq_pool == 0 || (L->seq_pool >= L->k && L->seq_pool <= Nc),
+                 SPTS_ERR_SHAPE, "%s: seq_pool must be 0 or in [k, Nc]", who);
     SPTS_REQUIRE(L->ltp_dout == 0 || (L->ltp_dout > 0 && L->ltp_dout % 256 == 0), SPTS_ERR_SHAPE,
                  "%s: ltp_dout must be 0 (= D) or a multiple of 256", who);
     const int dlow = L->ltp_dout > 0 ? L->ltp_dout : L->D;
@@ -229,7 +231,13 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   SPTS_TRY(launch_ltp_bf16(b.xn, Nc, D, W->ltp_a, L->r, W->ltp_b, L->ltp_dout > 0 ? L->ltp_dout : D, c, st, s,
                            L->ltp_top_m));
   SPTS_TRY(mark(12));
-  SPTS_TRY(launch_select_topk(sc, c, L->fuse, L->w_a, L->w_b, Nc, k, P, idx_f, f, nullptr, st, b.topk, s));
+  if (L->fuse == SPTS_FUSE_SEQUENTIAL) {
+    const int64_t pool = L->seq_pool > 0 ? L->seq_pool : std::min<int64_t>(Nc, 2 * k);
+    SPTS_TRY(launch_select_sequential(sc, c, Nc, pool, k, P, idx_f, b.topk, st, s));
+    SPTS_CUDA_TRY(cudaMemcpyAsync(f, c, static_cast<size_t>(Nc) * 4, cudaMemcpyDeviceToDevice, s));
+  } else {
+    SPTS_TRY(launch_select_topk(sc, c, L->fuse, L->w_a, L->w_b, Nc, k, P, idx_f, f, nullptr, st, b.topk, s));
+  }
   SPTS_TRY(launch_gather_rows(b.xn, Nc, idx_f, k, static_cast<int64_t>(D) * 2, b.xsel, nullptr, nullptr, st, s));
   SPTS_TRY(mark(13));
   GemmArgs g1{b.xsel, k, D, W->w_gate, W->w_up, L->F, SPTS_EPI_SWIGLU, b.act, nullptr, nullptr, 0.0, st};

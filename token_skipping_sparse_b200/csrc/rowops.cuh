@@ -32,6 +32,10 @@ spts_status launch_sum_groups(const float *group, int G, int64_t n, float *s, cu
 // grid when `scratch` (topk_scratch_bytes(Nc) bytes) is given and the
 // candidate set is large.
 size_t topk_scratch_bytes(int64_t Nc);
+size_t select_sequential_scratch_bytes(int64_t Nc);
+spts_status launch_select_sequential(const float *s_a, const float *s_b, int64_t Nc, int64_t k_pool, int64_t k,
+                                     int64_t force_tail, int32_t *idx_out, void *scratch, uint32_t *status,
+                                     cudaStream_t s);
 spts_status launch_select_topk(const float *s_a, const float *s_b, int mode, float w_a, float w_b, int64_t Nc,
                                int64_t k, int64_t force_tail, int32_t *idx_out, float *fused_out,
                                float *kth_out, uint32_t *status, void *scratch, cudaStream_t s);

@@ -42,14 +42,28 @@ struct FuseArgs {
   const float *sb;
   int mode;
   float wa, wb;
-  float ma, mb;  // maxima (MAXNORM_ADD)
+  float ma, mb;  // maxima (MAXNORM_ADD) or means (STD_ADD)
+  float da, db;  // standard deviations (STD_ADD)
 };
+
+// Mean and population standard deviation from fp64 sums, rounded to fp32.
+__device__ __forceinline__ void moments(double sum, double sumsq, int64_t n, float *mean, float *sd) {
+  const double mu = sum / static_cast<double>(n);
+  const double var = fmax(sumsq / static_cast<double>(n) - mu * mu, 0.0);
+  *mean = __double2float_rn(mu);
+  *sd = __double2float_rn(sqrt(var));
+}
 
 __device__ __forceinline__ float fused(const FuseArgs &f, int64_t i) {
   const float s = __ldg(f.sa + i);
   if (f.mode == SPTS_FUSE_NONE) return s;
   const float c = __ldg(f.sb + i);
   if (f.mode == SPTS_FUSE_MULTIPLY) return __fmul_rn(s, c);
+  if (f.mode == SPTS_FUSE_STD_ADD) {
+    const float ta = f.da > 0.f ? __fmul_rn(f.wa, __fdiv_rn(__fsub_rn(s, f.ma), f.da)) : 0.f;
+    const float tb = f.db > 0.f ? __fmul_rn(f.wb, __fdiv_rn(__fsub_rn(c, f.mb), f.db)) : 0.f;
+    return __fadd_rn(ta, tb);
+  }
   const float ta = f.ma > 0.f ? __fmul_rn(f.wa, __fdiv_rn(s, f.ma)) : 0.f;
   const float tb = f.mb > 0.f ? __fmul_rn(f.wb, __fdiv_rn(c, f.mb)) : 0.f;
   return __fadd_rn(ta, tb);
@@ -120,6 +134,32 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     }
     fa.ma = ma;
     fa.mb = mb;
+  }
+
+  // 1b. (STD_ADD) fp64 sums of both scores and their squares over all Nc
+  if (fa.mode == SPTS_FUSE_STD_ADD) {
+    __shared__ double dred[4][32];
+    double v[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int64_t i = tid; i < Nc; i += TK_THREADS) {
+      const double a = __ldg(fa.sa + i), b = __ldg(fa.sb + i);
+      v[0] += a;
+      v[1] += a * a;
+      v[2] += b;
+      v[3] += b * b;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v[q] += __shfl_xor_sync(0xffffffffu, v[q], o);
+      if (lane == 0) dred[q][w] = v[q];
+    }
+    __syncthreads();
+    double t[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int k2 = 0; k2 < 32; ++k2)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) t[q] += dred[q][k2];
+    moments(t[0], t[1], Nc, &fa.ma, &fa.da);
+    moments(t[2], t[3], Nc, &fa.mb, &fa.db);
   }
 
   // 2. fused scores, keys, fused_out, finiteness check
@@ -255,6 +295,7 @@ struct TopkScratch {
   uint32_t *keys;     // [n_free]
   uint32_t *hist;     // [TG_BINS]
   float *maxpart;     // [2][TG_MAX_CTAS]
+  double *sumpart;    // [4][TG_MAX_CTAS]: sums of s, s^2, c, c^2 (STD_ADD)
   uint32_t *chunk;    // [2][TG_MAX_CTAS]: per chunk, keys > T and keys == T
   uint32_t *sel;      // [4]: T, need_eq
 };
@@ -270,6 +311,8 @@ __host__ __device__ inline TopkScratch tg_carve(void *base, int64_t n_free) {
   p += tg_round(TG_BINS * 4);
   t.maxpart = reinterpret_cast<float *>(p);
   p += tg_round(2 * TG_MAX_CTAS * 4);
+  t.sumpart = reinterpret_cast<double *>(p);
+  p += tg_round(4 * TG_MAX_CTAS * 8);
   t.chunk = reinterpret_cast<uint32_t *>(p);
   p += tg_round(4 * TG_MAX_CTAS * 4);
   t.sel = reinterpret_cast<uint32_t *>(p);
@@ -281,8 +324,32 @@ __global__ void __launch_bounds__(TG_THREADS)
   __shared__ float red[2][32];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   for (int b = blockIdx.x * TG_THREADS + tid; b < TG_BINS; b += gridDim.x * TG_THREADS) t.hist[b] = 0u;
-  if (fa.mode != SPTS_FUSE_MAXNORM_ADD) return;
   const int64_t i0 = blockIdx.x * chunk, i1 = min(Nc, i0 + chunk);
+  if (fa.mode == SPTS_FUSE_STD_ADD) {
+    __shared__ double dred[4][32];
+    double v[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int64_t i = i0 + tid; i < i1; i += TG_THREADS) {
+      const double a = __ldg(fa.sa + i), b = __ldg(fa.sb + i);
+      v[0] += a;
+      v[1] += a * a;
+      v[2] += b;
+      v[3] += b * b;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v[q] += __shfl_xor_sync(0xffffffffu, v[q], o);
+      if (lane == 0) dred[q][w] = v[q];
+    }
+    __syncthreads();
+    if (tid < 4) {
+      double acc = 0.0;
+      for (int k2 = 0; k2 < 32; ++k2) acc += dred[tid][k2];
+      t.sumpart[tid * TG_MAX_CTAS + blockIdx.x] = acc;
+    }
+    return;
+  }
+  if (fa.mode != SPTS_FUSE_MAXNORM_ADD) return;
   float ma = -INFINITY, mb = -INFINITY;
   for (int64_t i = i0 + tid; i < i1; i += TG_THREADS) {
     ma = fmaxf(ma, __ldg(fa.sa + i));
@@ -334,11 +401,20 @@ __global__ void __launch_bounds__(TG_THREADS)
       if (lane == 0) mx[which] = m;
     }
   }
+  __shared__ double sums[4];
+  if (fa.mode == SPTS_FUSE_STD_ADD && tid < 4) {
+    double acc = 0.0;
+    for (int c = 0; c < n_cta; ++c) acc += t.sumpart[tid * TG_MAX_CTAS + c];  // fixed order
+    sums[tid] = acc;
+  }
   for (int b = tid; b < TG_BINS; b += TG_THREADS) h[b] = 0u;
   __syncthreads();
   if (fa.mode == SPTS_FUSE_MAXNORM_ADD) {
     fa.ma = mx[0];
     fa.mb = mx[1];
+  } else if (fa.mode == SPTS_FUSE_STD_ADD) {
+    moments(sums[0], sums[1], Nc, &fa.ma, &fa.da);
+    moments(sums[2], sums[3], Nc, &fa.mb, &fa.db);
   }
   const int64_t i0 = blockIdx.x * chunk, i1 = min(Nc, i0 + chunk);
   for (int64_t base = i0; base < i1; base += TG_THREADS) {
@@ -532,13 +608,13 @@ __global__ void __launch_bounds__(TG_THREADS)
 
 size_t topk_scratch_bytes(int64_t Nc) {
   return tg_round(static_cast<size_t>(Nc > 0 ? Nc : 1) * 4) + tg_round(TG_BINS * 4) + tg_round(2 * TG_MAX_CTAS * 4) +
-         tg_round(4 * TG_MAX_CTAS * 4) + 256;
+         tg_round(4 * TG_MAX_CTAS * 8) + tg_round(4 * TG_MAX_CTAS * 4) + 256;
 }
 
 spts_status launch_select_topk(const float *s_a, const float *s_b, int mode, float w_a, float w_b, int64_t Nc,
                                int64_t k, int64_t force_tail, int32_t *idx_out, float *fused_out,
                                float *kth_out, uint32_t *status, void *scratch, cudaStream_t s) {
-  FuseArgs fa{s_a, s_b, mode, w_a, w_b, 0.f, 0.f};
+  FuseArgs fa{s_a, s_b, mode, w_a, w_b, 0.f, 0.f, 0.f, 0.f};
   const int64_t n_free = Nc - force_tail;
   if (scratch != nullptr && n_free > TK_GRID_MIN) {
     const TopkScratch t = tg_carve(scratch, n_free);
@@ -579,6 +655,32 @@ spts_status launch_select_topk(const float *s_a, const float *s_b, int mode, flo
   }
   SPTS_CUDA_TRY(cudaGetLastError());
   return SPTS_OK;
+}
+
+size_t select_sequential_scratch_bytes(int64_t Nc) {
+  const size_t n = static_cast<size_t>(Nc > 0 ? Nc : 1) * 4;
+  return 3 * tg_round(n) + tg_round(topk_scratch_bytes(Nc));
+}
+
+// Sequential Select (Table D; reading): the pool = top-k_pool by s_a (tail
+// forced), then the top-k by s_b inside the pool (tail forced again), as
+// candidate indices ascending.  Three kernels of this file and two gathers.
+spts_status launch_select_sequential(const float *s_a, const float *s_b, int64_t Nc, int64_t k_pool, int64_t k,
+                                     int64_t force_tail, int32_t *idx_out, void *scratch, uint32_t *status,
+                                     cudaStream_t s) {
+  const size_t n = static_cast<size_t>(Nc > 0 ? Nc : 1) * 4;
+  uint8_t *p = static_cast<uint8_t *>(scratch);
+  int32_t *pool = reinterpret_cast<int32_t *>(p);
+  float *b_pool = reinterpret_cast<float *>(p + tg_round(n));
+  int32_t *local = reinterpret_cast<int32_t *>(p + 2 * tg_round(n));
+  void *tk = p + 3 * tg_round(n);
+  SPTS_TRY(launch_select_topk(s_a, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, Nc, k_pool, force_tail, pool, nullptr,
+                              nullptr, status, tk, s));
+  SPTS_TRY(launch_gather_i32(reinterpret_cast<const int32_t *>(s_b), pool, k_pool,
+                             reinterpret_cast<int32_t *>(b_pool), s));
+  SPTS_TRY(launch_select_topk(b_pool, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, k_pool, k, force_tail, local, nullptr,
+                              nullptr, status, tk, s));
+  return launch_gather_i32(pool, local, k, idx_out, s);
 }
 
 }  // namespace spts
