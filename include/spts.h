@@ -390,6 +390,24 @@ SPTS_API spts_status spts_msdp_forward(const spts_layer_desc *L, const spts_laye
                                        spts_stream stream);
 SPTS_API size_t spts_msdp_forward_workspace(const spts_layer_desc *L, int64_t N);
 
+/* A layer schedule of Table B (reading): layers [0, first_skip) are full
+ * layers over every token; stage st covers the layers up to stage_ends[st]
+ * and each of its layers selects k = min(budgets[st], |C|) active rows from
+ * the stage's candidates C; at a stage end the candidates are pruned to the
+ * top budgets[st] (after the last stage: the top after_last) by that
+ * layer's fused score, the last P always kept; the layers after the last
+ * stage are full layers over the survivors.  h [N, D] fp32 and pos [N] are
+ * compacted in place: *n_out rows remain.  sel_pos (nullable, sel_cap
+ * entries) receives, layer after layer, the positions of every skipping
+ * layer's attention set; sel_len [n_layers] their counts (0 for full
+ * layers).  W holds n_layers weight sets; F must be > 0; salience is off. */
+SPTS_API spts_status spts_schedule_forward(const spts_layer_desc *L, const spts_layer_weights *W, int n_layers,
+                                          int first_skip, const int *stage_ends, const int64_t *budgets,
+                                          int n_stages, int64_t after_last, float *h, int32_t *pos, int64_t N,
+                                          int64_t *n_out, int32_t *sel_pos, int64_t sel_cap, int64_t *sel_len,
+                                          void *ws, size_t ws_bytes, spts_stream stream);
+SPTS_API size_t spts_schedule_forward_workspace(const spts_layer_desc *L, int64_t N);
+
 #ifdef __cplusplus
 }
 #endif

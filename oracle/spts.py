@@ -43,7 +43,7 @@ __all__ = [
     "select_topk", "reduced_attention", "attention_residual", "reduced_ffn",
     "stage_prune", "inject_salience", "LayerWeights", "LayerConfig", "layer_forward",
     "msdp_forward", "MsdpConfig", "FUSE_NONE", "FUSE_MAXNORM_ADD", "FUSE_MULTIPLY", "FUSE_STD_ADD",
-    "FUSE_SEQUENTIAL", "select_sequential",
+    "FUSE_SEQUENTIAL", "select_sequential", "schedule_forward",
 ]
 
 FUSE_NONE = 0
@@ -485,3 +485,38 @@ def msdp_forward(h, pos, layers, mcfg: MsdpConfig, trace: list | None = None):
         pruned.append((pos[~keep_mask].copy(), h[~keep_mask].copy()))
         h, pos = h_new, pos_new
     return h, pos, pruned
+
+
+def schedule_forward(h, pos, layers, cfg: LayerConfig, first_skip, stage_ends, budgets, after_last,
+                     trace: list | None = None):
+    """A per-layer skipping schedule of Table B (reading).
+
+    Layers before ``first_skip`` are full layers (every token active).
+    Stage s runs the layers up to ``stage_ends[s]``; each selects
+    k = min(budgets[s], |C_s|) active rows from the stage's candidates C_s.
+    At a stage end the candidates are pruned to the top budgets[s] by that
+    layer's fused score (after the last stage to the top ``after_last``),
+    the probe tail kept; the layers after the last stage are full layers over
+    the survivors (Fig. A(c): skipped tokens are computed again later, pruned
+    ones are gone).  Returns (h of the survivors, their positions); ``trace``
+    receives per layer its k, its candidates' positions and the positions of
+    its attention set.
+    """
+    h = np.asarray(h, dtype=np.float64)
+    pos = np.asarray(pos)
+    stage = 0
+    for l, W in enumerate(layers):
+        Nc = h.shape[0]
+        skip = l >= first_skip and stage < len(stage_ends) and l <= stage_ends[stage]
+        k = min(budgets[stage], Nc) if skip else Nc
+        c = LayerConfig(**{**cfg.__dict__, "k": k, "salient_rows": None})
+        tr = {}
+        h, f = layer_forward(h, pos, W, c, tr)
+        if trace is not None:
+            trace.append(dict(layer=l, k=k, skip=skip, cand=pos.copy(), sel_pos=pos[tr["idx_attn"]], f=f))
+        if skip and l == stage_ends[stage]:
+            k_next = min(budgets[stage] if stage + 1 < len(stage_ends) else after_last, Nc)
+            kept, _ = select_topk(f, k_next, cfg.P)
+            h, pos = h[kept], pos[kept]
+            stage += 1
+    return h, pos

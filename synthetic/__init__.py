@@ -49,6 +49,8 @@ class Workload:
     ltp_dout: int = 0         # LTP proxy output channels (0: D)
     kv_active: bool = False   # reduced attention over the active rows' keys only
     ltp_top_m: int = 0        # LTP saliency = sum of the top m |y| (0: L2 norm)
+    # per-layer skipping schedule (first_skip, stage_ends, budgets, after_last); () for none
+    schedule: tuple = ()
 
     @property
     def k(self) -> int:
@@ -99,6 +101,17 @@ for _base in ("layer_32k", "layer_128k", "layer_small"):
     WORKLOADS[_base + "_std"] = replace(_w, name=_base + "_std", fuse=FUSE_STD_ADD)
     WORKLOADS[_base + "_seq"] = replace(_w, name=_base + "_seq", fuse=FUSE_SEQUENTIAL)
 del _base, _w
+# The 32-layer LLaMA-3.1-8B-shaped schedule of Table B (skipping in layers
+# 10..28, stages ending at 13/18/23/28 with budgets 9K/7K/4K/2K, 1K tokens
+# after) at Table 4's context lengths, with the pages' default settings: one
+# probe token, the Multiply fusion, the (D_low 512, r 192) proxy with top-rho
+# 0.2, and active-row keys in the skipping layers.  Random weights.
+for _n in (8, 16, 24, 32):
+    WORKLOADS[f"llama32_{_n}k"] = Workload(
+        f"llama32_{_n}k", N=_n * 1024, Hq=32, Hkv=8, d=128, P=1, keep="1", D=4096, F=14336, r=192,
+        fuse=FUSE_MULTIPLY, layers=32, seed=1200 + _n, ltp_dout=512, ltp_top_m=103, kv_active=True,
+        schedule=(10, (13, 18, 23, 28), (9 * 1024, 7 * 1024, 4 * 1024, 2 * 1024), 1024))
+del _n
 
 
 def _gen(seed):
@@ -146,26 +159,28 @@ def make_hidden(wl: Workload, n=None):
     return torch.randn(n, wl.D, generator=g, dtype=torch.float32).to(torch.bfloat16).float()
 
 
-def make_layer_weights(wl: Workload, layer: int = 0):
+def make_layer_weights(wl: Workload, layer: int = 0, device="cpu"):
     """bf16 weights of one Llama-shaped layer, nn.Linear layout, ~N(0, 0.02).
 
-    Keys: w_q [Hq*d, D], w_k / w_v [Hkv*d, D], w_o [D, Hq*d]; when F > 0 also
+    ``device`` draws them there (a different stream of values than on the
+    CPU: used where only timing needs them).  Keys: w_q [Hq*d, D], w_k / w_v [Hkv*d, D], w_o [D, Hq*d]; when F > 0 also
     w_gate / w_up [F, D], w_down [D, F], ltp_a [r, D], ltp_b [D_low, r] (D_low =
     ltp_dout, else D).  Norm
     weights are ones.
     """
-    g = _gen(wl.seed * 1000 + 17 + 101 * layer)
+    g = torch.Generator(device=device)
+    g.manual_seed(int(wl.seed * 1000 + 17 + 101 * layer))
     D, hd, kd = wl.D, wl.Hq * wl.d, wl.Hkv * wl.d
 
     def w(o, i):
-        return (0.02 * torch.randn(o, i, generator=g, dtype=torch.float32)).to(torch.bfloat16)
+        return (0.02 * torch.randn(o, i, generator=g, dtype=torch.float32, device=device)).to(torch.bfloat16)
 
     out = dict(w_q=w(hd, D), w_k=w(kd, D), w_v=w(kd, D), w_o=w(D, hd))
     if wl.F:
         out.update(w_gate=w(wl.F, D), w_up=w(wl.F, D), w_down=w(D, wl.F),
                    ltp_a=w(wl.r, D), ltp_b=w(wl.ltp_dout or D, wl.r))
-    out["norm_attn"] = torch.ones(D, dtype=torch.bfloat16)
-    out["norm_ffn"] = torch.ones(D, dtype=torch.bfloat16)
+    out["norm_attn"] = torch.ones(D, dtype=torch.bfloat16, device=device)
+    out["norm_ffn"] = torch.ones(D, dtype=torch.bfloat16, device=device)
     return out
 
 

@@ -250,3 +250,52 @@ def test_msdp_small_chain_matches_oracle():
     assert np.array_equal(pos_out.numpy(), opos)
     # eight layers of independently rounded stages on each side
     assert_close(h_out.numpy(), oh, 4 * LAYER_OUT_TOL, "msdp final hidden states")
+
+
+def test_dense_layer_path_is_bit_identical_to_the_selection_path():
+    # keep 1.0 without score outputs takes the dense path (no probe, LTP or
+    # selections); asking for the scores forces the general path
+    wl = WORKLOADS["layer_small"]
+    h = make_hidden(wl)
+    Wd = {n: t.cuda() for n, t in make_layer_weights(wl).items()}
+    pos = torch.arange(wl.N, dtype=torch.int32, device="cuda")
+    desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.N, fuse=wl.fuse)
+    h_fast = h.cuda()
+    S.spts_layer_forward(h_fast, pos, desc, Wd)
+    h_sel = h.cuda()
+    out = S.spts_layer_forward(h_sel, pos, desc, Wd, outputs=True)
+    S.check_device_status()
+    assert torch.equal(out["idx_attn"].cpu(), torch.arange(wl.N, dtype=torch.int32))
+    assert torch.equal(h_fast, h_sel)
+
+
+def test_schedule_small_matches_oracle():
+    # a Table-B-shaped schedule at small size: 2 full layers, three stages,
+    # two full layers over the survivors
+    wl = WORKLOADS["msdp_small"]
+    n_layers, first_skip, ends, budgets, after = 9, 2, (3, 5, 6), (450, 300, 200), 120
+    h = make_hidden(wl)
+    layers = [make_layer_weights(wl, i) for i in range(n_layers)]
+    desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, 0, fuse=wl.fuse)
+    hd = h.cuda()
+    pd = torch.arange(wl.N, dtype=torch.int32, device="cuda")
+    n, sel = S.spts_schedule_forward(hd, pd, desc, [{k: t.cuda() for k, t in W.items()} for W in layers], first_skip,
+                                     ends, budgets, after, selections=True)
+    S.check_device_status()
+    assert n == after
+    ow = [O.LayerWeights(**{k: _f64(t) for k, t in W.items()}) for W in layers]
+    cfg = O.LayerConfig(Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, P=wl.P, k=0, fuse=wl.fuse)
+    tr = []
+    oh, opos = O.schedule_forward(h.numpy().astype(np.float64), np.arange(wl.N), ow, cfg, first_skip, ends, budgets,
+                                  after, tr)
+    # layer by layer: the attention sets agree until a legitimate near-tie split
+    for l, t in enumerate(tr):
+        if not t["skip"]:
+            assert sel[l] is None
+            continue
+        g = sel[l].cpu().numpy()
+        assert len(g) == t["k"]
+        if not np.array_equal(g, t["sel_pos"]):
+            return   # the chains diverge from here on (checked per call elsewhere)
+    assert np.array_equal(pd[:n].cpu().numpy(), opos)
+    assert_close(hd[:n].cpu().numpy(), oh, 4 * LAYER_OUT_TOL, "schedule final hidden states")

@@ -414,6 +414,29 @@ def test_msdp_all_ratios_one_is_dense_stack_and_sets_nest():
     assert set(opos.tolist()) == seen and {pos[-1], pos[-2]} <= seen
 
 
+def test_schedule_without_skipping_is_the_dense_stack_and_sets_nest():
+    # budgets and the final count at least N: every layer is a full layer
+    h, pos, W0, cfg = _tiny_layer(N=40, P=2)
+    layers = [W0] + [_tiny_layer(N=40, P=2)[2] for _ in range(5)]
+    out, opos = O.schedule_forward(h, pos, layers, cfg, 1, (2, 4), (40, 50), 40)
+    want = h
+    for W in layers:
+        want = _dense_layer_torch(want, pos, W, cfg)
+    np.testing.assert_allclose(out, want, rtol=1e-10, atol=1e-10)
+    assert np.array_equal(opos, pos)
+    # with budgets: k per layer, candidate sets nest, the tail survives
+    tr = []
+    out, opos = O.schedule_forward(h, pos, layers, cfg, 1, (2, 4), (30, 20), 10, tr)
+    assert [t["k"] for t in tr] == [40, 30, 30, 20, 20, 10]
+    assert [len(t["cand"]) for t in tr] == [40, 40, 40, 30, 30, 10]
+    assert [t["skip"] for t in tr] == [False, True, True, True, True, False]
+    for t in tr:
+        assert set(t["sel_pos"]) <= set(t["cand"]) and set(pos[-2:]) <= set(t["sel_pos"])
+    for a, b in zip(tr, tr[1:]):
+        assert set(b["cand"]) <= set(a["cand"])
+    assert np.array_equal(opos, tr[-1]["cand"]) and out.shape == (10, h.shape[1])
+
+
 # ---------------------------------------------------------------- synthetic salience
 def test_inject_salience_closed_form():
     # two probes x two heads of one KV group: mean (0.5, 0.5, 0, 0) -> unit (1, 1, 0, 0)/sqrt(2)

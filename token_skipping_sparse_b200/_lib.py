@@ -33,7 +33,7 @@ EXPORTS = (
     "spts_reduced_attention_workspace", "spts_reduced_ffn", "spts_reduced_ffn_workspace", "spts_stage_prune",
     "spts_stage_prune_workspace", "spts_stage_prune_noalloc", "spts_rmsnorm_rows", "spts_rope", "spts_gather_rows", "spts_linear",
     "spts_linear_workspace", "spts_inject_salience", "spts_layer_forward", "spts_layer_forward_workspace",
-    "spts_msdp_forward", "spts_msdp_forward_workspace",
+    "spts_msdp_forward", "spts_msdp_forward_workspace", "spts_schedule_forward", "spts_schedule_forward_workspace",
 )
 
 
@@ -128,6 +128,10 @@ if hasattr(lib, "spts_layer_forward"):
     _sig("spts_msdp_forward", i32, [C.POINTER(LayerDesc), C.POINTER(LayerWeights), i32, i32, C.POINTER(C.c_int64),
                                     i32, vp, vp, i64, vp, vp, sz, vp])
     _sig("spts_msdp_forward_workspace", sz, [C.POINTER(LayerDesc), i64])
+_sig("spts_schedule_forward", i32, [C.POINTER(LayerDesc), C.POINTER(LayerWeights), i32, i32, C.POINTER(C.c_int),
+                                    C.POINTER(C.c_int64), i32, i64, vp, vp, i64, C.POINTER(C.c_int64), vp, i64,
+                                    C.POINTER(C.c_int64), vp, sz, vp])
+_sig("spts_schedule_forward_workspace", sz, [C.POINTER(LayerDesc), i64])
 
 
 # ---------------------------------------------------------------- helpers
@@ -436,3 +440,37 @@ def spts_msdp_forward(h, pos, desc, layer_weights_list, layers_per_stage, stage_
         out.append(sp[off:off + int(k)])
         off += int(k)
     return int(stage_k[-1]), out
+
+
+def spts_schedule_forward(h, pos, desc, layer_weights_list, first_skip, stage_ends, budgets, after_last,
+                          selections=False, ws=None):
+    """A Table-B layer schedule over h [N, D] fp32 and pos [N] int32, in place.
+
+    Returns the number of rows left (h[:n], pos[:n] hold them); with
+    ``selections`` also the per-layer positions of every skipping layer's
+    attention set (None for full layers)."""
+    N = h.shape[0]
+    n_layers = len(layer_weights_list)
+    Ws = (LayerWeights * n_layers)(*[layer_weights(w) for w in layer_weights_list])
+    ends = (C.c_int * len(stage_ends))(*stage_ends)
+    buds = (C.c_int64 * len(budgets))(*budgets)
+    n_out = C.c_int64(0)
+    sel = sel_len = None
+    cap = 0
+    if selections:
+        cap = sum(min(b, N) for b in budgets) * n_layers
+        sel = torch.empty(cap, dtype=torch.int32, device=h.device)
+        sel_len = (C.c_int64 * n_layers)()
+    n = lib.spts_schedule_forward_workspace(C.byref(desc), N)
+    ws = workspace(n) if ws is None else ws
+    check(lib.spts_schedule_forward(C.byref(desc), Ws, n_layers, first_skip, ends, buds, len(stage_ends), after_last,
+                                    ptr(h), ptr(pos), N, C.byref(n_out), ptr(sel) if sel is not None else None, cap,
+                                    sel_len, ptr(ws), ws.numel(), stream_ptr()))
+    if not selections:
+        return int(n_out.value)
+    out, off = [], 0
+    for l in range(n_layers):
+        m = int(sel_len[l])
+        out.append(sel[off:off + m] if m else None)
+        off += m
+    return int(n_out.value), out

@@ -100,6 +100,51 @@ spts_status check_layer(const spts_layer_desc *L, const spts_layer_weights *W, i
   return SPTS_OK;
 }
 
+// keep 1.0 (k == Nc) with no score outputs asked for and no planted salience:
+// every selection is the identity, so the layer is the dense Llama layer --
+// no probe, no LTP, no selections, no gathers.
+spts_status dense_layer(const spts_layer_desc *L, const spts_layer_weights *W, float *h, const int32_t *pos,
+                        int64_t Nc, const spts_layer_outputs &o, const LayerBufs &b, uint32_t *st, cudaStream_t s) {
+  const int D = L->D, hq = L->Hq * L->d, hk = L->Hkv * L->d;
+  const float scale = 1.0f / sqrtf(static_cast<float>(L->d));
+  void *osel = o.o_sel ? o.o_sel : b.osel;
+  auto mark = [&](int i) -> spts_status {
+    if (o.stage_events != nullptr) SPTS_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(o.stage_events[i]), s));
+    return SPTS_OK;
+  };
+  SPTS_TRY(mark(0));
+  SPTS_TRY(launch_rmsnorm_rows(h, nullptr, Nc, D, W->norm_attn, L->eps, b.xn, s));
+  SPTS_TRY(mark(1));
+  GemmArgs gk{b.xn, Nc, D, W->w_k, nullptr, hk, SPTS_EPI_ROPE, b.kk, nullptr, pos, L->theta, st};
+  SPTS_TRY(launch_gemm(gk, s));
+  SPTS_TRY(mark(2));
+  GemmArgs gv{b.xn, Nc, D, W->w_v, nullptr, hk, SPTS_EPI_STORE, b.vv, nullptr, nullptr, 0.0, st};
+  SPTS_TRY(launch_gemm(gv, s));
+  for (int i = 3; i <= 7; ++i) SPTS_TRY(mark(i));
+  GemmArgs gq{b.xn, Nc, D, W->w_q, nullptr, hq, SPTS_EPI_ROPE, b.qsel, nullptr, pos, L->theta, st};
+  SPTS_TRY(launch_gemm(gq, s));
+  SPTS_TRY(mark(8));
+  SPTS_TRY(launch_attention_bf16(b.qsel, pos, Nc, b.kk, b.vv, pos, Nc, L->Hq, L->Hkv, scale, osel, st, s));
+  SPTS_TRY(mark(9));
+  SPTS_TRY(launch_iota_i32(b.idx_a, Nc, s));
+  GemmArgs go{osel, Nc, hq, W->w_o, nullptr, D, SPTS_EPI_SCATTER_ADD, h, b.idx_a, nullptr, 0.0, st};
+  SPTS_TRY(launch_gemm(go, s));
+  if (o.h_attn) SPTS_CUDA_TRY(cudaMemcpyAsync(o.h_attn, h, static_cast<size_t>(Nc) * D * 4, cudaMemcpyDeviceToDevice, s));
+  SPTS_TRY(mark(10));
+  if (L->F <= 0) {
+    for (int i = 11; i < SPTS_LAYER_STAGE_EVENTS; ++i) SPTS_TRY(mark(i));
+    return SPTS_OK;
+  }
+  SPTS_TRY(launch_rmsnorm_rows(h, nullptr, Nc, D, W->norm_ffn, L->eps, b.xn, s));
+  for (int i = 11; i <= 13; ++i) SPTS_TRY(mark(i));
+  GemmArgs g1{b.xn, Nc, D, W->w_gate, W->w_up, L->F, SPTS_EPI_SWIGLU, b.act, nullptr, nullptr, 0.0, st};
+  SPTS_TRY(launch_gemm(g1, s));
+  SPTS_TRY(mark(14));
+  GemmArgs g2{b.act, Nc, L->F, W->w_down, nullptr, D, SPTS_EPI_SCATTER_ADD, h, b.idx_a, nullptr, 0.0, st};
+  SPTS_TRY(launch_gemm(g2, s));
+  return mark(15);
+}
+
 }  // namespace
 
 extern "C" {
@@ -126,6 +171,8 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   carve(cv, L, Nc, b);
   uint32_t *st = cv.status();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (L->k == Nc && !o.s && !o.c && !o.f && !o.idx_attn && !o.idx_ffn && L->n_salient == 0)
+    return dense_layer(L, W, h, pos, Nc, o, b, st, s);
   const int D = L->D, P = L->P, hq = L->Hq * L->d, hk = L->Hkv * L->d;
   const int64_t k = L->k;
   float *sc = o.s ? o.s : b.s;
@@ -319,6 +366,99 @@ spts_status spts_msdp_forward(const spts_layer_desc *L, const spts_layer_weights
     SPTS_CUDA_TRY(cudaMemcpyAsync(h, ha, static_cast<size_t>(Nc) * L->D * 4, cudaMemcpyDeviceToDevice, s));
     SPTS_CUDA_TRY(cudaMemcpyAsync(pos, pa, static_cast<size_t>(Nc) * 4, cudaMemcpyDeviceToDevice, s));
   }
+  return SPTS_OK;
+}
+
+// ---------------------------------------------------------------- layer schedule
+size_t spts_schedule_forward_workspace(const spts_layer_desc *L, int64_t N) {
+  if (L == nullptr || N <= 0) return kStatusBytes;
+  spts_layer_desc l = *L;
+  l.k = N;
+  const size_t lw = Carver::round(spts_layer_forward_workspace(&l, N));
+  return lw + Carver::round(static_cast<size_t>(N) * L->D * 4) + 4 * Carver::round(static_cast<size_t>(N) * 4);
+}
+
+spts_status spts_schedule_forward(const spts_layer_desc *L, const spts_layer_weights *W, int n_layers, int first_skip,
+                                  const int *stage_ends, const int64_t *budgets, int n_stages, int64_t after_last,
+                                  float *h, int32_t *pos, int64_t N, int64_t *n_out, int32_t *sel_pos,
+                                  int64_t sel_cap, int64_t *sel_len, void *ws, size_t ws_bytes, spts_stream stream) {
+  const char *who = "spts_schedule_forward";
+  SPTS_REQUIRE(L && W && stage_ends && budgets && h && pos && n_out, SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(n_stages >= 1 && n_layers >= 1 && first_skip >= 0 && first_skip <= stage_ends[0] &&
+                   stage_ends[n_stages - 1] < n_layers,
+               SPTS_ERR_SHAPE, "%s: need first_skip <= stage_ends[0] and stage_ends[last] < n_layers", who);
+  for (int st = 0; st < n_stages; ++st) {
+    SPTS_REQUIRE(st == 0 || stage_ends[st] > stage_ends[st - 1], SPTS_ERR_SHAPE, "%s: stage ends must ascend", who);
+    SPTS_REQUIRE(budgets[st] >= L->P, SPTS_ERR_SHAPE, "%s: every budget must be >= P", who);
+  }
+  SPTS_REQUIRE(after_last >= L->P, SPTS_ERR_SHAPE, "%s: after_last must be >= P", who);
+  SPTS_REQUIRE(L->F > 0, SPTS_ERR_SHAPE, "%s: pruning uses the fused FFN score, so F must be > 0", who);
+  SPTS_REQUIRE(sel_pos == nullptr || sel_len != nullptr, SPTS_ERR_INVALID, "%s: sel_pos needs sel_len", who);
+  SPTS_TRY(check_ws(ws, ws_bytes, spts_schedule_forward_workspace(L, N), who));
+  spts_layer_desc lmax = *L;
+  lmax.k = N;
+  const size_t lw = Carver::round(spts_layer_forward_workspace(&lmax, N));
+  char *extra = static_cast<char *>(ws) + lw;
+  float *h2 = reinterpret_cast<float *>(extra);
+  extra += Carver::round(static_cast<size_t>(N) * L->D * 4);
+  int32_t *pos2 = reinterpret_cast<int32_t *>(extra);
+  extra += Carver::round(static_cast<size_t>(N) * 4);
+  float *f = reinterpret_cast<float *>(extra);
+  extra += Carver::round(static_cast<size_t>(N) * 4);
+  int32_t *kept = reinterpret_cast<int32_t *>(extra);
+  extra += Carver::round(static_cast<size_t>(N) * 4);
+  int32_t *idx_a = reinterpret_cast<int32_t *>(extra);
+  uint32_t *st = static_cast<uint32_t *>(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  float *ha = h, *hb = h2;
+  int32_t *pa = pos, *pb = pos2;
+  int64_t Nc = N, sel_off = 0;
+  int stage = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    const bool skip = l >= first_skip && stage < n_stages && l <= stage_ends[stage];
+    spts_layer_desc d = *L;
+    d.n_salient = 0;
+    d.salient_rows = nullptr;
+    spts_layer_outputs o;
+    memset(&o, 0, sizeof(o));
+    if (sel_len) sel_len[l] = 0;
+    if (!skip) {  // a full layer over the current tokens (the dense path)
+      d.k = Nc;
+      SPTS_TRY(spts_layer_forward(&d, &W[l], ha, pa, Nc, &o, ws, lw, stream));
+      continue;
+    }
+    d.k = std::min<int64_t>(budgets[stage], Nc);
+    const bool stage_end = l == stage_ends[stage];
+    o.idx_attn = idx_a;
+    if (stage_end) o.f = f;
+    SPTS_TRY(spts_layer_forward(&d, &W[l], ha, pa, Nc, &o, ws, lw, stream));
+    if (sel_pos) {  // positions of this layer's attention set (consecutive-layer overlap diagnostics)
+      SPTS_REQUIRE(sel_off + d.k <= sel_cap, SPTS_ERR_SHAPE, "%s: sel_pos holds %lld positions, needs more", who,
+                   static_cast<long long>(sel_cap));
+      SPTS_TRY(launch_gather_i32(pa, idx_a, d.k, sel_pos + sel_off, s));
+      sel_len[l] = d.k;
+      sel_off += d.k;
+    }
+    if (stage_end) {  // prune: the next stage's candidates (after the last: the tokens kept)
+      const int64_t k_next = std::min<int64_t>(stage + 1 < n_stages ? budgets[stage] : after_last, Nc);
+      Carver lcv(ws, lw);  // the layers are done with their workspace: its top-k scratch serves the prune
+      LayerBufs lb;
+      carve(lcv, &lmax, N, lb);
+      SPTS_TRY(launch_select_topk(f, nullptr, SPTS_FUSE_NONE, 0.f, 0.f, Nc, k_next, L->P, kept, nullptr, nullptr, st,
+                                  lb.topk, s));
+      SPTS_TRY(launch_gather_rows(ha, Nc, kept, k_next, static_cast<int64_t>(L->D) * 4, hb, pa, pb, st, s));
+      std::swap(ha, hb);
+      std::swap(pa, pb);
+      Nc = k_next;
+      ++stage;
+    }
+  }
+  if (ha != h) {
+    SPTS_CUDA_TRY(cudaMemcpyAsync(h, ha, static_cast<size_t>(Nc) * L->D * 4, cudaMemcpyDeviceToDevice, s));
+    SPTS_CUDA_TRY(cudaMemcpyAsync(pos, pa, static_cast<size_t>(Nc) * 4, cudaMemcpyDeviceToDevice, s));
+  }
+  *n_out = Nc;
   return SPTS_OK;
 }
 

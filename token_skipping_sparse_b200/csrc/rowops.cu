@@ -281,6 +281,20 @@ spts_status launch_sum_groups(const float *group, int G, int64_t n, float *s, cu
 
 namespace spts {
 
+// dst[i] = i.
+__global__ void iota_i32_kernel(int32_t *__restrict__ dst, int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = static_cast<int32_t>(i);
+}
+
+spts_status launch_iota_i32(int32_t *dst, int64_t n, cudaStream_t s) {
+  if (n == 0) return SPTS_OK;
+  iota_i32_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(dst, n);
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
 // dst[i] = src[idx[i]] for int32 vectors (positions of the selected rows).
 __global__ void gather_i32_kernel(const int32_t *__restrict__ src, const int32_t *__restrict__ idx, int64_t m,
                                   int32_t *__restrict__ dst) {

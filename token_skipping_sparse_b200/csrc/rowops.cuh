@@ -26,6 +26,7 @@ spts_status launch_inject_salience(void *k, int64_t Nc, const void *q_probe, int
                                    const int32_t *rows, int64_t n_rows, float shift, uint32_t *status,
                                    cudaStream_t s);
 spts_status launch_gather_i32(const int32_t *src, const int32_t *idx, int64_t m, int32_t *dst, cudaStream_t s);
+spts_status launch_iota_i32(int32_t *dst, int64_t n, cudaStream_t s);
 spts_status launch_sum_groups(const float *group, int G, int64_t n, float *s, cudaStream_t st);
 
 // Top-k selection: radix select + stable compaction, on one CTA, or on the
