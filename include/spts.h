@@ -281,8 +281,9 @@ SPTS_API spts_status spts_linear(const void *A, int64_t M, int K, const void *W,
 SPTS_API size_t spts_linear_workspace(void);
 
 /* Adds shift * unit(mean of the group's probe queries) to K[rows[t], g] for
- * every KV head g (K bf16 [Nc, Hkv, d], q_probe bf16 [P, Hq, d]).  This is a
- * synthetic-workload step that plants salient keys; it is not part of SPTS. */
+ * every KV head g (K bf16 [Nc, Hkv, d], q_probe bf16 [P, Hq, d]); rows must
+ * be distinct.  This is a synthetic-workload step that plants salient keys;
+ * it is not part of SPTS. */
 SPTS_API spts_status spts_inject_salience(void *k, int64_t Nc, const void *q_probe, int P, int Hq, int Hkv, int d,
                                  const int32_t *rows, int64_t n_rows, float shift, spts_stream stream);
 

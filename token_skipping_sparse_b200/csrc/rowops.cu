@@ -235,14 +235,28 @@ __global__ void inject_salience_kernel(__nv_bfloat16 *__restrict__ k, int64_t Nc
     __syncthreads();
   }
   const float u = mean / sqrtf(red[0]);
-  for (int64_t t = t_begin; t < t_end; ++t) {
-    const int32_t row = rows[t];
-    if (row < 0 || row >= Nc) {
-      if (i == 0) raise_status(status, SPTS_DEV_BADINDEX, 0x62u, static_cast<uint32_t>(row));
-      continue;
+  // eight rows at a time: their index and element loads are all in flight
+  // together instead of one dependent round trip per row
+  constexpr int B = 8;
+  for (int64_t t0 = t_begin; t0 < t_end; t0 += B) {
+    int32_t row[B];
+    float v[B];
+#pragma unroll
+    for (int j = 0; j < B; ++j) row[j] = t0 + j < t_end ? rows[t0 + j] : -1;
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      const bool ok = row[j] >= 0 && row[j] < Nc;
+      v[j] = ok ? __bfloat162float(k[(static_cast<int64_t>(row[j]) * Hkv + g) * d + i]) : 0.f;
     }
-    __nv_bfloat16 *kr = k + (static_cast<int64_t>(row) * Hkv + g) * d;
-    kr[i] = __float2bfloat16_rn(__bfloat162float(kr[i]) + shift * u);
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      if (t0 + j >= t_end) break;
+      if (row[j] < 0 || row[j] >= Nc) {
+        if (i == 0) raise_status(status, SPTS_DEV_BADINDEX, 0x62u, static_cast<uint32_t>(row[j]));
+        continue;
+      }
+      k[(static_cast<int64_t>(row[j]) * Hkv + g) * d + i] = __float2bfloat16_rn(v[j] + shift * u);
+    }
   }
 }
 
