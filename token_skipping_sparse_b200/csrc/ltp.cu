@@ -11,9 +11,10 @@
 //            epilogue warps fold every chunk into a per-row sum of squares.
 // With top_m > 0 (D_low = Dout <= 512, both chunks resident in TMEM) the
 // score is instead the sum of the top_m largest |y| of the row (top-rho
-// channel saliency, Table E): each row's thread finds its top_m-th largest
-// |y| by a bitwise search over the float bits (31 counting passes over the
-// row in TMEM), then sums the values above it plus the ties it needs.
+// channel saliency, Table E): each row's thread searches the float bits of
+// |y| from the top for a threshold with exactly top_m values at or above it
+// (counting passes over the row in TMEM, at most 31, usually about half),
+// then sums the values above it plus the ties at it that top_m needs.
 // Per row only 2*D bytes of X are read from HBM; A and B (2 x r x D bf16)
 // are shared by all CTAs through L2.  Waits are bounded.
 #include "host.hpp"
@@ -194,21 +195,27 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok) {
         tc_fence_after();
-        // largest T with at least top_m values of |y| >= T (|y| bits order as uints)
+        // a T with exactly top_m values of |y| >= T, or else the top_m-th
+        // largest |y| itself: bit by bit from the top (|y| bits order as
+        // uints), stopping once exactly top_m values lie at or above T
         uint32_t T = 0u;
+        int at_or_above = p.Dout;  // values >= T
 #pragma unroll 1
-        for (int b = 30; b >= 0; --b) {
+        for (int b = 30; b >= 0 && __any_sync(0xffffffffu, at_or_above != p.top_m); --b) {
           const uint32_t cand = T | (1u << b);
           int cnt = 0;
 #pragma unroll 1
           for (int c0 = 0; c0 < p.Dout; c0 += 32) {
             uint32_t y[32];
-            tmem_ld32(lane_base + c0, y);
+            tmem_ld32(lane_base + c0, y);  // warp-wide: every lane loads, finished ones included
             tmem_ld_wait();
 #pragma unroll
             for (int t = 0; t < 32; ++t) cnt += (y[t] & 0x7FFFFFFFu) >= cand;
           }
-          if (cnt >= p.top_m) T = cand;
+          if (at_or_above != p.top_m && cnt >= p.top_m) {
+            T = cand;
+            at_or_above = cnt;
+          }
         }
         int gt = 0;
 #pragma unroll 1
