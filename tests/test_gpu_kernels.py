@@ -199,6 +199,23 @@ def test_reduced_ffn_small():
     assert_close(got, want, 2e-2, "reduced ffn")
 
 
+# ---------------------------------------------------------------- synthetic salience
+@pytest.mark.parametrize("Nc,Hq,Hkv,d,P,n_rows", [(3000, 32, 8, 128, 64, 655), (500, 4, 4, 64, 16, 10),
+                                                  (700, 32, 8, 128, 1, 129), (300, 8, 2, 128, 128, 1)])
+def test_inject_salience_matches_oracle(Nc, Hq, Hkv, d, P, n_rows):
+    # several row chunks per KV head with a ragged last chunk, fewer query
+    # vectors than slices (P = 1), and a single row
+    k = torch.randn(Nc, Hkv, d).to(torch.bfloat16)
+    q = torch.randn(P, Hq, d).to(torch.bfloat16)
+    rows = np.sort(rng.choice(Nc, n_rows, replace=False)).astype(np.int32)
+    kd = k.cuda()
+    S.spts_inject_salience(kd, q.cuda(), torch.from_numpy(rows).cuda(), 3.0)
+    want = O.inject_salience(np64(k), np64(q), rows, 3.0, Hkv)
+    got = np64(kd)
+    assert np.array_equal(np.delete(got, rows, axis=0), np.delete(np64(k), rows, axis=0))
+    assert_bf16_close(got, want, 0.0, "salient keys")
+
+
 # ---------------------------------------------------------------- bounded waits
 def test_bounded_wait_timeout_reports_and_context_survives():
     A = torch.randn(512, 4096).to(torch.bfloat16).cuda()

@@ -7,8 +7,10 @@
 // two consecutive Q tiles, A and B, so every K/V tile it loads feeds four
 // M=128 MMAs (S and PV for each tile) and the softmax of one tile runs while
 // the tensor core works on the other.
-//   warp 0      TMA: both Q tiles once, then K and V tiles of 128 keys into
-//               a 2-stage ring (128-byte swizzle);
+//   warp 0      TMA: both Q tiles once (issued at entry, while warps 0..3
+//               find the tiles' key ranges by warp-wide searches), then K
+//               and V tiles of 128 keys into a 2-stage ring (128-byte
+//               swizzle);
 //   warp 1      MMA, per key tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).
 //               S_X = Q_X K^T lands in TMEM region S_X; the softmax writes
 //               bf16 P over it and PV reads P from TMEM (A operand in TMEM)
@@ -16,7 +18,8 @@
 //   warps 2..3  idle (they complete warpgroup 0 for the register split);
 //   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B, one thread
 //               per Q row: tcgen05.ld of the S row, causal mask (only on key
-//               tiles crossing the tile's diagonal), row max with independent
+//               tiles crossing the tile's diagonal, against the row's last
+//               visible key found once up front), row max with independent
 //               three-input max accumulators, lazy O rescale (only when the
 //               running max grows by more than 2^8), the scale folded into a
 //               packed fp32x2 FFMA before exp2, row sums in packed fp32x2
@@ -92,16 +95,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-__device__ __forceinline__ int upper_bound(const int32_t *a, int n, int32_t v) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (a[mid] <= v) lo = mid + 1;
-    else hi = mid;
-  }
-  return lo;
-}
-
 __global__ void __launch_bounds__(THREADS, 1)
     attention_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
@@ -140,17 +133,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // both Q tiles are in flight while the key ranges are searched
+    mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
     for (int x = 0; x < 2; ++x) {
-      const int first = t0 + x * p.tq;
-      if (first < p.m) {
-        const int last = min(first + p.tq, p.m) - 1;
-        s_range[2 * x] = upper_bound(p.kpos, p.Nc, p.qpos[last]);
-        s_range[2 * x + 1] = upper_bound(p.kpos, p.Nc, p.qpos[first]);
-      } else {
-        s_range[2 * x] = 0;  // tile B beyond the last token: no work
-        s_range[2 * x + 1] = 0;
-      }
+      tma_load_3d(sQ + x * TILE_BYTES, &tmQ, q_full, 0, g * p.G, t0 + x * p.tq);
+      tma_load_3d(sQ + x * TILE_BYTES + CHUNK_BYTES, &tmQ, q_full, 64, g * p.G, t0 + x * p.tq);
     }
+  }
+  // Key ranges of the two tiles, one warp-wide search each on warps 0..3:
+  // kv_end[X] = keys at or before the tile's last query, mask_from[X] = keys
+  // at or before its first (a tile beyond the last token has no work).
+  if (warp < 4) {
+    const int x = warp >> 1, first = t0 + x * p.tq;
+    int r = 0;
+    if (first < p.m) r = warp_upper_bound(p.kpos, p.Nc, p.qpos[(warp & 1) ? first : min(first + p.tq, p.m) - 1]);
+    if (lane == 0) s_range[2 * x + (warp & 1)] = r;
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, TMEM_COLS);
@@ -167,14 +164,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
-      for (int x = 0; x < 2; ++x) {
-        tma_load_3d(sQ + x * TILE_BYTES, &tmQ, q_full, 0, g * p.G, t0 + x * p.tq);
-        tma_load_3d(sQ + x * TILE_BYTES + CHUNK_BYTES, &tmQ, q_full, 64, g * p.G, t0 + x * p.tq);
-      }
       uint32_t issued = 0, issued_par = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % KV_STAGES;
@@ -265,6 +256,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool valid = tok < p.m;
     const int32_t qp = valid ? p.qpos[tok] : INT_MIN;
     const int kv_end = s_range[2 * x], mask_from = s_range[2 * x + 1];
+    // This row sees keys [0, lim): kpos ascending, so lim = keys at or before
+    // its query, between the tile's mask_from and kv_end (0 for padding rows).
+    // Found once here, while the first S tile is on its way.
+    int lim = 0;
+    if (valid) {
+      int lo = mask_from, hi = kv_end;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(p.kpos + mid) <= qp) lo = mid + 1;
+        else hi = mid;
+      }
+      lim = lo;
+    }
     const int n_tiles = x == 0 ? n_a : n_b;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const uint32_t s_col = x * BKV, o_col = 256 + x * 128;
@@ -284,13 +288,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld32(lane_base + s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32 * c));
       tmem_ld_wait();
       const int j0 = j * BKV;
-      const bool need_mask = (j0 + BKV > mask_from) || (j0 + BKV > kv_end);
-      if (need_mask) {
+      // causal mask, only on key tiles past the tile's first query (which
+      // includes every tile reaching past kv_end >= mask_from)
+      if (j0 + BKV > mask_from) {
+        const int vis = lim - j0;
 #pragma unroll
-        for (int c = 0; c < BKV; ++c) {
-          const int key = j0 + c;
-          if (!(key < kv_end && __ldg(p.kpos + key) <= qp)) xr[c] = 0xff800000u;  // -inf
-        }
+        for (int c = 0; c < BKV; ++c)
+          if (c >= vis) xr[c] = 0xff800000u;  // -inf
       }
       float m8[8];
 #pragma unroll

@@ -53,25 +53,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// Number of a[0..n) that are <= v (a sorted ascending), by the whole warp:
-// each step samples 32 evenly spaced points, so 2^17 keys take 4 dependent
-// loads instead of 17.
-__device__ __forceinline__ int warp_upper_bound(const int32_t *a, int n, int32_t v) {
-  const int lane = threadIdx.x & 31;
-  int lo = 0, hi = n;  // answer in [lo, hi]
-  while (lo < hi) {
-    const int step = (hi - lo + 31) >> 5;
-    const int idx = lo + (lane + 1) * step - 1;
-    const bool le = idx < hi && __ldg(a + idx) <= v;
-    const int cnt = __popc(__ballot_sync(0xffffffffu, le));  // samples 0..cnt-1 are <= v
-    const int nlo = lo + cnt * step;
-    const int nhi = lo + (cnt + 1) * step - 1;
-    lo = nlo;
-    if (nhi < hi) hi = nhi;
-  }
-  return lo;
-}
-
 // Work item (local key tile i, sub-item u) uses TMEM buffer (i & 1) * 2 + (u & 1)
 // and consumer warpgroup i & 1.  Uses of that buffer before this item:
 __device__ __forceinline__ uint32_t buffer_uses(int i, int u, int nsub) {

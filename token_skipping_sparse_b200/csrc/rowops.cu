@@ -213,44 +213,69 @@ spts_status launch_gather_rows(const void *src, int64_t n_src, const int32_t *ro
 
 // ---------------------------------------------------------------- salience
 // Synthetic-workload step (not SPTS): K[rows[t], g] += shift * unit(mean of
-// the group's probe queries).  Blocks (KV head, chunk of SAL_ROWS rows), d
-// threads; each block recomputes the group mean (a few KB of reads).
-constexpr int SAL_ROWS = 16;
+// the group's probe queries).  Blocks (KV head, chunk of SAL_ROWS rows) of
+// SAL_THREADS threads = S slices of d threads (d a power of two <= 1024).
+// Each block recomputes the group mean: slice s sums the query vectors
+// s, s + S, ... with eight loads in flight per thread, in fp64, where the sum
+// of bf16 values is exact, so the slice order does not change it.  Slice s
+// then updates rows t_begin + s, + S, ... (rows must be distinct).
+constexpr int SAL_ROWS = 64;
+constexpr int SAL_THREADS = 1024;
+constexpr int SAL_BATCH = 8;
 
-__global__ void inject_salience_kernel(__nv_bfloat16 *__restrict__ k, int64_t Nc, const __nv_bfloat16 *__restrict__ q,
-                                       int P, int Hq, int Hkv, int d, const int32_t *__restrict__ rows, int64_t n_rows,
-                                       float shift, uint32_t *status) {
-  extern __shared__ float red[];
-  const int g = blockIdx.x, i = threadIdx.x, G = Hq / Hkv;
-  const int64_t t_begin = static_cast<int64_t>(blockIdx.y) * SAL_ROWS;
-  const int64_t t_end = t_begin + SAL_ROWS < n_rows ? t_begin + SAL_ROWS : n_rows;
+__global__ void __launch_bounds__(SAL_THREADS)
+    inject_salience_kernel(__nv_bfloat16 *__restrict__ k, int64_t Nc, const __nv_bfloat16 *__restrict__ q, int P,
+                           int Hq, int Hkv, int d, const int32_t *__restrict__ rows, int64_t n_rows, float shift,
+                           uint32_t *status) {
+  extern __shared__ double part[];                          // [S][d] partial sums
+  float *red = reinterpret_cast<float *>(part + SAL_THREADS);  // [d] squares, then [d] means
+  float *meanv = red + d;
+  const int g = blockIdx.x, G = Hq / Hkv, S = SAL_THREADS / d;
+  const int i = static_cast<int>(threadIdx.x) % d, sl = static_cast<int>(threadIdx.x) / d;
+  const int n = P * G;
   double acc = 0.0;
-  for (int p = 0; p < P; ++p)
-    for (int j = 0; j < G; ++j) acc += __bfloat162float(q[(static_cast<int64_t>(p) * Hq + g * G + j) * d + i]);
-  const float mean = static_cast<float>(acc / (P * G));
-  red[i] = mean * mean;
+  for (int pg0 = sl; pg0 < n; pg0 += SAL_BATCH * S) {
+    float v[SAL_BATCH];
+#pragma unroll
+    for (int u = 0; u < SAL_BATCH; ++u) {
+      const int pg = pg0 + u * S;
+      v[u] = pg < n ? __bfloat162float(q[(static_cast<int64_t>(pg / G) * Hq + g * G + pg % G) * d + i]) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < SAL_BATCH; ++u) acc += v[u];
+  }
+  part[sl * d + i] = acc;
   __syncthreads();
-  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
-    if (i < o) red[i] += red[i + o];
+  if (sl == 0) {
+    double t = 0.0;
+    for (int j = 0; j < S; ++j) t += part[j * d + i];
+    const float mean = static_cast<float>(t / n);
+    meanv[i] = mean;
+    red[i] = mean * mean;
+  }
+  __syncthreads();
+  for (int o = d / 2; o > 0; o >>= 1) {
+    if (sl == 0 && i < o) red[i] += red[i + o];
     __syncthreads();
   }
-  const float u = mean / sqrtf(red[0]);
-  // eight rows at a time: their index and element loads are all in flight
+  const float u = meanv[i] / sqrtf(red[0]);
+  const int64_t t_begin = static_cast<int64_t>(blockIdx.y) * SAL_ROWS;
+  const int64_t t_end = t_begin + SAL_ROWS < n_rows ? t_begin + SAL_ROWS : n_rows;
+  // SAL_BATCH rows per pass: their index and element loads are all in flight
   // together instead of one dependent round trip per row
-  constexpr int B = 8;
-  for (int64_t t0 = t_begin; t0 < t_end; t0 += B) {
-    int32_t row[B];
-    float v[B];
+  for (int64_t t0 = t_begin + sl; t0 < t_end; t0 += static_cast<int64_t>(SAL_BATCH) * S) {
+    int32_t row[SAL_BATCH];
+    float v[SAL_BATCH];
 #pragma unroll
-    for (int j = 0; j < B; ++j) row[j] = t0 + j < t_end ? rows[t0 + j] : -1;
+    for (int j = 0; j < SAL_BATCH; ++j) row[j] = t0 + j * S < t_end ? rows[t0 + j * S] : -1;
 #pragma unroll
-    for (int j = 0; j < B; ++j) {
+    for (int j = 0; j < SAL_BATCH; ++j) {
       const bool ok = row[j] >= 0 && row[j] < Nc;
       v[j] = ok ? __bfloat162float(k[(static_cast<int64_t>(row[j]) * Hkv + g) * d + i]) : 0.f;
     }
 #pragma unroll
-    for (int j = 0; j < B; ++j) {
-      if (t0 + j >= t_end) break;
+    for (int j = 0; j < SAL_BATCH; ++j) {
+      if (t0 + j * S >= t_end) break;
       if (row[j] < 0 || row[j] >= Nc) {
         if (i == 0) raise_status(status, SPTS_DEV_BADINDEX, 0x62u, static_cast<uint32_t>(row[j]));
         continue;
@@ -265,9 +290,10 @@ spts_status launch_inject_salience(void *k, int64_t Nc, const void *q_probe, int
                                    cudaStream_t s) {
   if (n_rows == 0) return SPTS_OK;
   const dim3 grid(static_cast<unsigned>(Hkv), static_cast<unsigned>((n_rows + SAL_ROWS - 1) / SAL_ROWS));
-  inject_salience_kernel<<<grid, d, d * sizeof(float), s>>>(static_cast<__nv_bfloat16 *>(k), Nc,
-                                                           static_cast<const __nv_bfloat16 *>(q_probe), P, Hq,
-                                                           Hkv, d, rows, n_rows, shift, status);
+  const size_t smem = SAL_THREADS * sizeof(double) + 2 * static_cast<size_t>(d) * sizeof(float);
+  inject_salience_kernel<<<grid, SAL_THREADS, smem, s>>>(static_cast<__nv_bfloat16 *>(k), Nc,
+                                                         static_cast<const __nv_bfloat16 *>(q_probe), P, Hq, Hkv,
+                                                         d, rows, n_rows, shift, status);
   note_launch();
   SPTS_CUDA_TRY(cudaGetLastError());
   return SPTS_OK;
