@@ -89,7 +89,24 @@ def _layer_case(name):
                                   "layer_small_dlow", "layer_small_rho", "layer_small_std", "layer_small_seq"])
 def test_layer_small_matches_oracle(name):
     wl, h, W, sal, pos = _layer_case(name)
-    Wd = {n: t.cuda() for n, t in W.items()}
+    _check_layer(wl, h, W, sal, pos, {n: t.cuda() for n, t in W.items()})
+
+
+# Non-unit norm weights, distinct for the two norms (the FFN input is a full
+# RMSNorm pass over h') or one shared vector (only the attention rows are
+# renormalised, in place).
+@pytest.mark.parametrize("shared", [False, True])
+def test_layer_norm_weights(shared):
+    wl, h, W, sal, pos = _layer_case("layer_small")
+    g = torch.Generator().manual_seed(11)
+    W["norm_attn"] = (1 + 0.2 * torch.randn(wl.D, generator=g)).to(torch.bfloat16)
+    W["norm_ffn"] = W["norm_attn"] if shared else (1 + 0.2 * torch.randn(wl.D, generator=g)).to(torch.bfloat16)
+    Wd = {n: t.cuda() for n, t in W.items() if n != "norm_ffn"}
+    Wd["norm_ffn"] = Wd["norm_attn"] if shared else W["norm_ffn"].cuda()
+    _check_layer(wl, h, W, sal, pos, Wd)
+
+
+def _check_layer(wl, h, W, sal, pos, Wd):
     desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k, fuse=wl.fuse,
                         salient_rows=sal.cuda(), salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m, seq_pool=0,
                         kv_active_only=wl.kv_active)

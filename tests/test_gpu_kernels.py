@@ -205,15 +205,19 @@ def test_reduced_ffn_small():
 def test_inject_salience_matches_oracle(Nc, Hq, Hkv, d, P, n_rows):
     # several row chunks per KV head with a ragged last chunk, fewer query
     # vectors than slices (P = 1), and a single row
-    k = torch.randn(Nc, Hkv, d).to(torch.bfloat16)
-    q = torch.randn(P, Hq, d).to(torch.bfloat16)
-    rows = np.sort(rng.choice(Nc, n_rows, replace=False)).astype(np.int32)
+    g = torch.Generator().manual_seed(Nc + P)
+    k = torch.randn(Nc, Hkv, d, generator=g).to(torch.bfloat16)
+    q = torch.randn(P, Hq, d, generator=g).to(torch.bfloat16)
+    rows = np.sort(np.random.default_rng(Nc).choice(Nc, n_rows, replace=False)).astype(np.int32)
     kd = k.cuda()
     S.spts_inject_salience(kd, q.cuda(), torch.from_numpy(rows).cuda(), 3.0)
     want = O.inject_salience(np64(k), np64(q), rows, 3.0, Hkv)
     got = np64(kd)
     assert np.array_equal(np.delete(got, rows, axis=0), np.delete(np64(k), rows, axis=0))
-    assert_bf16_close(got, want, 0.0, "salient keys")
+    # the kernel forms k + shift*u in fp32 (|k| + shift <~ 8): its rounding
+    # error, below 2^-20, decides the result only where the sum cancels to
+    # near zero; elsewhere within one bf16 ulp of the fp64 oracle
+    assert_bf16_close(got, want, 2.0 ** -20, "salient keys")
 
 
 # ---------------------------------------------------------------- bounded waits

@@ -7,10 +7,10 @@
 // two consecutive Q tiles, A and B, so every K/V tile it loads feeds four
 // M=128 MMAs (S and PV for each tile) and the softmax of one tile runs while
 // the tensor core works on the other.
-//   warp 0      TMA: both Q tiles once (issued at entry, while warps 0..3
-//               find the tiles' key ranges by warp-wide searches), then K
-//               and V tiles of 128 keys into a 2-stage ring (128-byte
-//               swizzle);
+//   warp 0      TMA: both Q tiles and key tile 0 at entry (while warps 0..3
+//               find the tiles' key ranges by warp-wide searches), then the
+//               other K and V tiles of 128 keys into a 2-stage ring
+//               (128-byte swizzle);
 //   warp 1      MMA, per key tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).
 //               S_X = Q_X K^T lands in TMEM region S_X; the softmax writes
 //               bf16 P over it and PV reads P from TMEM (A operand in TMEM)
@@ -133,12 +133,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // both Q tiles are in flight while the key ranges are searched
+    // both Q tiles and key tile 0 (where every tile's key loop starts) are
+    // in flight while the key ranges are searched
     mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
     for (int x = 0; x < 2; ++x) {
       tma_load_3d(sQ + x * TILE_BYTES, &tmQ, q_full, 0, g * p.G, t0 + x * p.tq);
       tma_load_3d(sQ + x * TILE_BYTES + CHUNK_BYTES, &tmQ, q_full, 64, g * p.G, t0 + x * p.tq);
     }
+    mbar_arrive_expect_tx(&k_full[0], TILE_BYTES);
+    tma_load_3d(sK, &tmK, &k_full[0], 0, g, 0);
+    tma_load_3d(sK + CHUNK_BYTES, &tmK, &k_full[0], 64, g, 0);
+    mbar_arrive_expect_tx(&v_full[0], TILE_BYTES);
+    tma_load_3d(sV, &tmV, &v_full[0], 0, g, 0);
+    tma_load_3d(sV + CHUNK_BYTES, &tmV, &v_full[0], 64, g, 0);
   }
   // Key ranges of the two tiles, one warp-wide search each on warps 0..3:
   // kv_end[X] = keys at or before the tile's last query, mask_from[X] = keys
@@ -164,10 +171,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
     if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      uint32_t issued = 0, issued_par = 0;
-      for (int j = 0; j < n_kv; ++j) {
+      uint32_t issued = 1u, issued_par = 0;  // stage 0: key tile 0, loaded at entry
+      for (int j = 1; j < n_kv; ++j) {
         const int st = j % KV_STAGES;
         const uint32_t ph = (j / KV_STAGES) & 1;
         if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_flag, p.status, p.wait_ns, 0x21u)) break;
@@ -179,6 +184,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_3d(sV + st * TILE_BYTES + CHUNK_BYTES, &tmV, &v_full[st], 64, g, j * BKV);
         issued |= 1u << st;
         issued_par = (issued_par & ~(1u << st)) | (ph << st);
+      }
+      if (n_kv == 0) {  // no visible key: let the entry loads of tile 0 land
+        mbar_drain(&k_full[0], 0, p.status);
+        mbar_drain(&v_full[0], 0, p.status);
       }
       if (*abort_flag) {
         mbar_drain(q_full, 0, p.status);

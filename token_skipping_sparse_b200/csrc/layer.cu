@@ -273,7 +273,13 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   float *c = o.c ? o.c : b.c;
   float *f = o.f ? o.f : b.f;
   int32_t *idx_f = o.idx_ffn ? o.idx_ffn : b.idx_f;
-  SPTS_TRY(launch_rmsnorm_rows(h, nullptr, Nc, D, W->norm_ffn, L->eps, b.xn, s));
+  // xn is free again: RMSNorm(h') under the FFN norm goes there.  When both
+  // norms share one weight vector (or have none), RMSNorm(h') differs from
+  // the attention input only on the k attention rows: renormalise just those.
+  if (W->norm_ffn == W->norm_attn)
+    SPTS_TRY(launch_rmsnorm_rows(h, idx_a, k, D, W->norm_ffn, L->eps, b.xn, s, /*scatter=*/true));
+  else
+    SPTS_TRY(launch_rmsnorm_rows(h, nullptr, Nc, D, W->norm_ffn, L->eps, b.xn, s));
   SPTS_TRY(mark(11));
   SPTS_TRY(launch_ltp_bf16(b.xn, Nc, D, W->ltp_a, L->r, W->ltp_b, L->ltp_dout > 0 ? L->ltp_dout : D, c, st, s,
                            L->ltp_top_m));

@@ -11,15 +11,37 @@
 namespace spts {
 
 // ---------------------------------------------------------------- RMSNorm
-// One warp per output row; x fp32 [*, D], y bf16 [m, D].  D % 8 == 0.
+// One warp per row; x fp32 [*, D], y bf16.  Row i reads x[rows[i]] (x[i]
+// without rows) and writes y[i], or y[rows[i]] when `scatter` (renormalise
+// some rows in place).  D % 8 == 0.
+__device__ __forceinline__ uint4 norm8(const float (&v)[8], float inv, const __nv_bfloat16 *w, int c) {
+  float o[8];
+  if (w) {
+    uint4 wv = __ldg(reinterpret_cast<const uint4 *>(w) + c);
+    const __nv_bfloat16 *wb = reinterpret_cast<const __nv_bfloat16 *>(&wv);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) o[t] = v[t] * inv * __bfloat162float(wb[t]);
+  } else {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) o[t] = v[t] * inv;
+  }
+  uint4 r;
+  r.x = pack_bf16x2(o[0], o[1]);
+  r.y = pack_bf16x2(o[2], o[3]);
+  r.z = pack_bf16x2(o[4], o[5]);
+  r.w = pack_bf16x2(o[6], o[7]);
+  return r;
+}
+
 __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const float *__restrict__ x,
                                                            const int32_t *__restrict__ rows, int64_t m, int D,
                                                            const __nv_bfloat16 *__restrict__ w, float eps,
-                                                           __nv_bfloat16 *__restrict__ y) {
+                                                           __nv_bfloat16 *__restrict__ y, int scatter) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (i >= m) return;
   const int lane = threadIdx.x & 31;
   const int64_t src = rows ? rows[i] : i;
+  const int64_t dst = scatter ? src : i;
   const float4 *xr = reinterpret_cast<const float4 *>(x + src * D);
   float ss = 0.f;
   for (int c = lane; c < D / 4; c += 32) {
@@ -29,25 +51,11 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const float *__restri
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float inv = 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
-  uint4 *yr = reinterpret_cast<uint4 *>(y + i * D);
+  uint4 *yr = reinterpret_cast<uint4 *>(y + dst * D);
   for (int c = lane; c < D / 8; c += 32) {
     float4 a = __ldg(xr + 2 * c), b = __ldg(xr + 2 * c + 1);
-    float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    if (w) {
-      uint4 wv = __ldg(reinterpret_cast<const uint4 *>(w) + c);
-      const __nv_bfloat16 *wb = reinterpret_cast<const __nv_bfloat16 *>(&wv);
-#pragma unroll
-      for (int t = 0; t < 8; ++t) v[t] = v[t] * inv * __bfloat162float(wb[t]);
-    } else {
-#pragma unroll
-      for (int t = 0; t < 8; ++t) v[t] = v[t] * inv;
-    }
-    uint4 o;
-    o.x = pack_bf16x2(v[0], v[1]);
-    o.y = pack_bf16x2(v[2], v[3]);
-    o.z = pack_bf16x2(v[4], v[5]);
-    o.w = pack_bf16x2(v[6], v[7]);
-    yr[c] = o;
+    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    yr[c] = norm8(v, inv, w, c);
   }
 }
 
@@ -57,12 +65,13 @@ template <int V8>
 __global__ void __launch_bounds__(256) rmsnorm_rows_reg_kernel(const float *__restrict__ x,
                                                                const int32_t *__restrict__ rows, int64_t m,
                                                                const __nv_bfloat16 *__restrict__ w, float eps,
-                                                               __nv_bfloat16 *__restrict__ y) {
+                                                               __nv_bfloat16 *__restrict__ y, int scatter) {
   constexpr int D = 256 * V8;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (i >= m) return;
   const int lane = threadIdx.x & 31;
   const int64_t src = rows ? rows[i] : i;
+  const int64_t dst = scatter ? src : i;
   const float4 *xr = reinterpret_cast<const float4 *>(x + src * D);
   float4 a[V8], b[V8];
 #pragma unroll
@@ -83,49 +92,28 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_reg_kernel(const float *__re
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   const float inv = 1.0f / sqrtf(s / static_cast<float>(D) + eps);
-  uint4 *yr = reinterpret_cast<uint4 *>(y + i * D);
+  uint4 *yr = reinterpret_cast<uint4 *>(y + dst * D);
 #pragma unroll
   for (int t = 0; t < V8; ++t) {
     const int c = lane + 32 * t;
-    float v[8] = {a[t].x, a[t].y, a[t].z, a[t].w, b[t].x, b[t].y, b[t].z, b[t].w};
-    if (w) {
-      uint4 wv = __ldg(reinterpret_cast<const uint4 *>(w) + c);
-      const __nv_bfloat16 *wb = reinterpret_cast<const __nv_bfloat16 *>(&wv);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = v[e] * inv * __bfloat162float(wb[e]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = v[e] * inv;
-    }
-    uint4 o;
-    o.x = pack_bf16x2(v[0], v[1]);
-    o.y = pack_bf16x2(v[2], v[3]);
-    o.z = pack_bf16x2(v[4], v[5]);
-    o.w = pack_bf16x2(v[6], v[7]);
-    yr[c] = o;
+    const float v[8] = {a[t].x, a[t].y, a[t].z, a[t].w, b[t].x, b[t].y, b[t].z, b[t].w};
+    yr[c] = norm8(v, inv, w, c);
   }
 }
 
 spts_status launch_rmsnorm_rows(const float *x, const int32_t *rows, int64_t m, int D, const void *w, float eps,
-                                void *y, cudaStream_t s) {
+                                void *y, cudaStream_t s, bool scatter) {
   if (m == 0) return SPTS_OK;
-  const int64_t blocks = (m + 7) / 8;
+  const unsigned blocks = static_cast<unsigned>((m + 7) / 8);
   const __nv_bfloat16 *wb = static_cast<const __nv_bfloat16 *>(w);
   __nv_bfloat16 *yb = static_cast<__nv_bfloat16 *>(y);
-  if (D == 4096) {
-    rmsnorm_rows_reg_kernel<16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, rows, m, wb, eps, yb);
-    note_launch();
-    SPTS_CUDA_TRY(cudaGetLastError());
-    return SPTS_OK;
-  }
-  if (D == 1024) {
-    rmsnorm_rows_reg_kernel<4><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, rows, m, wb, eps, yb);
-    note_launch();
-    SPTS_CUDA_TRY(cudaGetLastError());
-    return SPTS_OK;
-  }
-  rmsnorm_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-      x, rows, m, D, static_cast<const __nv_bfloat16 *>(w), eps, static_cast<__nv_bfloat16 *>(y));
+  const int sc = scatter ? 1 : 0;
+  if (D == 4096)
+    rmsnorm_rows_reg_kernel<16><<<blocks, 256, 0, s>>>(x, rows, m, wb, eps, yb, sc);
+  else if (D == 1024)
+    rmsnorm_rows_reg_kernel<4><<<blocks, 256, 0, s>>>(x, rows, m, wb, eps, yb, sc);
+  else
+    rmsnorm_rows_kernel<<<blocks, 256, 0, s>>>(x, rows, m, D, wb, eps, yb, sc);
   note_launch();
   SPTS_CUDA_TRY(cudaGetLastError());
   return SPTS_OK;

@@ -16,8 +16,10 @@ struct RopeFreqs {
 };
 void fill_rope_freqs(RopeFreqs *f, int d, double theta);
 
+// Row i of x (x[rows[i]] with rows) normalised into y[i] (y[rows[i]] when
+// scatter).
 spts_status launch_rmsnorm_rows(const float *x, const int32_t *rows, int64_t m, int D, const void *w, float eps,
-                                void *y, cudaStream_t s);
+                                void *y, cudaStream_t s, bool scatter = false);
 spts_status launch_rope(void *x, int64_t m, int H, int d, const int32_t *pos, double theta, cudaStream_t s);
 spts_status launch_gather_rows(const void *src, int64_t n_src, const int32_t *rows, int64_t m, int64_t row_bytes,
                                void *dst, const int32_t *pos_in, int32_t *pos_out, uint32_t *status,
