@@ -31,7 +31,12 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 48 KB
 constexpr int GROUP_M = 16;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+// Scatter-add staging: per epilogue warp 32 rows x 32 fp32, rows padded to
+// 36 words so that the row-per-thread writes and the row-segment reads of
+// 16-byte vectors are both free of bank conflicts.
+constexpr int STG_STRIDE = 36;
+constexpr int STG_BYTES = 4 * 32 * STG_STRIDE * 4;   // 18 KB
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + STG_BYTES;
 
 struct Params {
   int M, N, K;         // N: output columns of W (for SWIGLU: of W_gate and of W_up each)
@@ -69,21 +74,13 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float *v
   }
 }
 
-// Angle pos * inv_freq reduced to [-pi, pi] in fp64; the fast sine/cosine of
-// the reduced fp32 angle is accurate to ~1e-6, far below bf16 resolution.
-__device__ __forceinline__ void rope_angle_f(int32_t pos, double inv_freq, float *c, float *s) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double inv_two_pi = 0.15915494309189533576888376337251;
-  double a = static_cast<double>(pos) * inv_freq;
-  a = fma(-two_pi, rint(a * inv_two_pi), a);
-  __sincosf(static_cast<float>(a), s, c);
-}
 
 // Fused epilogue of one 256-column accumulator tile for the 32 rows this warp
 // owns: `tbase` addresses the warp's TMEM lanes at the tile's first column;
 // `row` is this thread's output row, `tn` the tile's column index.
 template <int EPI>
-__device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, int64_t row, bool live, int tn) {
+__device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, int64_t row, bool live, int tn,
+                                              float *stg) {
   if (EPI == SPTS_EPI_STORE) {
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
 #pragma unroll 1
@@ -101,7 +98,7 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
       // one angle per pair, shared by the tile's heads (same row position)
       float cs[32], sn[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) rope_angle_f(pos, p.freqs.inv_freq[c * 32 + i], &cs[i], &sn[i]);
+      for (int i = 0; i < 32; ++i) rope_cos_sin(pos, p.freqs, c * 32 + i, &cs[i], &sn[i]);
 #pragma unroll 1
       for (int hc = 0; hc < BN / 128; ++hc) {   // heads of 128 columns in this tile
         uint32_t lo[32], hi[32];
@@ -135,23 +132,42 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
       for (int i = 0; i < 32; ++i) y[i] = silu(__uint_as_float(g[i])) * __uint_as_float(u[i]);
       if (live) store_bf16x32(out + row * p.N + tn * 128 + c * 32, y);
     }
-  } else {  // SCATTER_ADD into fp32 rows: rows are unique, so one vector reduction per 4 columns
-           // performs the single fp32 add h + acc in L2 without a load round trip
+  } else {  // SCATTER_ADD into fp32 rows (unique rows): each 32-column chunk of the warp's 32 rows goes
+           // through shared memory so that 8 lanes update one row's 128 contiguous bytes: coalesced
+           // loads and stores instead of 32 scattered half-sector reductions per instruction
     float *out = static_cast<float *>(p.out);
-    const int64_t orow = live ? p.rows[row] : 0;
+    const int lane = threadIdx.x & 31;
+    const int64_t orow = live ? p.rows[row] : -1;
+    int64_t dst[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = __shfl_sync(0xffffffffu, orow, 4 * i + (lane >> 3));
+    float4 *srow = reinterpret_cast<float4 *>(stg + lane * STG_STRIDE);
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       uint32_t r[32];
       tmem_ld32(tbase + c * 32, r);
       tmem_ld_wait();
-      if (live) {
-        float *dst = out + orow * p.N + tn * BN + c * 32;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * q), "r"(r[4 * q + 0]),
-                       "r"(r[4 * q + 1]), "r"(r[4 * q + 2]), "r"(r[4 * q + 3])
-                       : "memory");
-      }
+      for (int q = 0; q < 8; ++q)
+        srow[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                              __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+      __syncwarp();
+      float4 hv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (dst[i] >= 0)
+          hv[i] = reinterpret_cast<const float4 *>(out + dst[i] * p.N + tn * BN + c * 32)[lane & 7];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (dst[i] >= 0) {
+          const float4 v = reinterpret_cast<const float4 *>(stg + (4 * i + (lane >> 3)) * STG_STRIDE)[lane & 7];
+          hv[i].x += v.x;
+          hv[i].y += v.y;
+          hv[i].z += v.z;
+          hv[i].w += v.w;
+          reinterpret_cast<float4 *>(out + dst[i] * p.N + tn * BN + c * 32)[lane & 7] = hv[i];
+        }
+      __syncwarp();
     }
   }
 }
@@ -276,6 +292,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // epilogue warps 2..5 -> TMEM lane quadrant warp % 4
     const int quad = warp & 3;
     const int row_in_tile = quad * 32 + lane;
+    float *stg = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256) + (warp - 2) * 32 * STG_STRIDE;
     int local = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -288,7 +305,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int64_t row = static_cast<int64_t>(tm) * BM + row_in_tile;
       const bool live = row < p.M;
       const uint32_t tbase = tmem_addr(tmem_base, quad * 32, acc * BN);
-      epilogue_rows<EPI>(p, tbase, row, live, tn);
+      epilogue_rows<EPI>(p, tbase, row, live, tn, stg);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
@@ -336,7 +353,7 @@ constexpr int STAGES2 = 6;
 constexpr int HALF_BYTES = 128 * BK * 2;       // 16 KB: 128 rows x 64 bf16
 constexpr int STAGE2_BYTES = 2 * HALF_BYTES;   // one CTA's A half + B half
 constexpr int GROUP_M2 = 8;                    // 256-row tiles per raster group
-constexpr size_t SMEM2_BYTES = 1024 + STAGES2 * STAGE2_BYTES + 256;
+constexpr size_t SMEM2_BYTES = 1024 + STAGES2 * STAGE2_BYTES + 256 + STG_BYTES;
 
 __device__ __forceinline__ void tile_coords2(int t, int tiles_m2, int tiles_n, int &tm, int &tn) {
   const int per_group = GROUP_M2 * tiles_n;
@@ -459,6 +476,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     const int quad = warp & 3;
     const int row_in_tile = quad * 32 + lane;
+    float *stg = reinterpret_cast<float *>(smem + STAGES2 * STAGE2_BYTES + 256) + (warp - 2) * 32 * STG_STRIDE;
     int local = 0;
     for (int t = pair; t < tiles; t += n_pairs, ++local) {
       const int acc = local & 1;
@@ -471,7 +489,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int64_t row = static_cast<int64_t>(tm) * 256 + rank * 128 + row_in_tile;
       const bool live = row < p.M;
       const uint32_t tbase = tmem_addr(tmem_base, quad * 32, acc * BN);
-      epilogue_rows<EPI>(p, tbase, row, live, tn);
+      epilogue_rows<EPI>(p, tbase, row, live, tn, stg);
       tc_fence_before();
       mbar_arrive_remote(&tempty[acc], 0);
     }

@@ -120,17 +120,8 @@ spts_status launch_rmsnorm_rows(const float *x, const int32_t *rows, int64_t m, 
 }
 
 // ---------------------------------------------------------------- RoPE
-// Angle pos * inv_freq[i] is formed and reduced modulo 2*pi in fp64, then the
-// fast sine/cosine runs on the reduced fp32 angle (error ~1e-6 for positions
-// up to 2^31).  One thread per (row, pair i), looping over the heads.
-__device__ __forceinline__ void rope_angle(int32_t pos, double inv_freq, float *c, float *s) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double inv_two_pi = 0.15915494309189533576888376337251;
-  double a = static_cast<double>(pos) * inv_freq;
-  a = fma(-two_pi, rint(a * inv_two_pi), a);
-  __sincosf(static_cast<float>(a), s, c);
-}
-
+// Rotate-half RoPE with the angles of rope_cos_sin (reduced in turns, error
+// ~1e-6).  One thread per (row, pair i), looping over the heads.
 __global__ void rope_kernel(__nv_bfloat16 *__restrict__ x, int64_t m, int H, int d,
                             const int32_t *__restrict__ pos, RopeFreqs f) {
   const int half = d / 2;
@@ -139,7 +130,7 @@ __global__ void rope_kernel(__nv_bfloat16 *__restrict__ x, int64_t m, int H, int
   const int64_t row = t / half;
   const int i = static_cast<int>(t % half);
   float c, s;
-  rope_angle(pos[row], f.inv_freq[i], &c, &s);
+  rope_cos_sin(pos[row], f, i, &c, &s);
   __nv_bfloat16 *xr = x + row * static_cast<int64_t>(H) * d;
   for (int h = 0; h < H; ++h) {
     const float x1 = __bfloat162float(xr[h * d + i]);
@@ -150,7 +141,12 @@ __global__ void rope_kernel(__nv_bfloat16 *__restrict__ x, int64_t m, int H, int
 }
 
 void fill_rope_freqs(RopeFreqs *f, int d, double theta) {
-  for (int i = 0; i < d / 2 && i < 128; ++i) f->inv_freq[i] = pow(theta, -2.0 * i / d);
+  for (int i = 0; i < d / 2 && i < 128; ++i) {
+    f->inv_freq[i] = pow(theta, -2.0 * i / d);
+    const double g = f->inv_freq[i] / 6.283185307179586476925286766559;
+    f->turn_hi[i] = static_cast<float>(g);
+    f->turn_lo[i] = static_cast<float>(g - static_cast<double>(f->turn_hi[i]));
+  }
 }
 
 spts_status launch_rope(void *x, int64_t m, int H, int d, const int32_t *pos, double theta, cudaStream_t s) {

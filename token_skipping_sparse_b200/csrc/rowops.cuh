@@ -13,8 +13,31 @@ namespace spts {
 
 struct RopeFreqs {
   double inv_freq[128];  // theta^(-2i/d), i < d/2
+  // the same frequencies in turns (inv_freq / 2 pi) as two fp32 parts:
+  // turn_hi = fp32(g), turn_lo = fp32(g - turn_hi), about 2^-24 g
+  float turn_hi[128], turn_lo[128];
 };
 void fill_rope_freqs(RopeFreqs *f, int d, double theta);
+
+// cos and sin of pos * inv_freq[i].  The angle is reduced in turns without
+// fp64 arithmetic: pos * turn_hi = hi + lo exactly (an FMA two-product; pos
+// below 2^24 is exact in fp32), the integer part of hi is dropped exactly
+// and pos * turn_lo adds the next 24 bits of the frequency, so the reduced
+// angle is within ~1e-7 turns; __sincosf then works on [-pi, pi] where its
+// error is ~2^-21.  Positions from 2^24 on take an fp64 reduction.
+__device__ __forceinline__ void rope_cos_sin(int32_t pos, const RopeFreqs &f, int i, float *c, float *s) {
+  float t;
+  if (pos < (1 << 24)) {
+    const float pf = static_cast<float>(pos);
+    const float hi = pf * f.turn_hi[i];
+    const float lo = fmaf(pf, f.turn_hi[i], -hi);
+    t = (hi - rintf(hi)) + (lo + pf * f.turn_lo[i]);
+  } else {
+    const double a = static_cast<double>(pos) * (static_cast<double>(f.turn_hi[i]) + f.turn_lo[i]);
+    t = static_cast<float>(a - rint(a));
+  }
+  __sincosf(t * 6.28318530717958647692f, s, c);
+}
 
 // Row i of x (x[rows[i]] with rows) normalised into y[i] (y[rows[i]] when
 // scatter).
