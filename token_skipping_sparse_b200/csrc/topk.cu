@@ -24,10 +24,11 @@ constexpr int TK_THREADS = 1024;
 constexpr int TK_ITEMS = 8;
 constexpr int TK_SMEM_KEYS = 49152;  // 192 KB of cached keys
 // Above this many free candidates the grid path runs (given scratch).
-// Measured: at 8K candidates one CTA takes 15 us and the grid 26 us; at 32K
-// one CTA 29-38 us and the grid 27-32 us; at 128K 147-316 us against 53-60.
+// Measured inside the 32K layer: one CTA 34 / 66 us for the two selections,
+// the grid 42 / 82 us (its five launches cost more than they save there);
+// at 128K one CTA 147-316 us against 53-60 us for the grid.
 #ifndef TK_GRID_MIN
-#define TK_GRID_MIN 24576
+#define TK_GRID_MIN 49152
 #endif
 
 __device__ __forceinline__ uint32_t order_key(float f) {
