@@ -267,13 +267,15 @@ def gpu_arm(args, rank, world, dev):
     idx = torch.empty(ldesc.k, dtype=torch.int32, device=dev)
     evs = S.stage_events()
     S.spts_layer_forward(hb, lcase.pos, ldesc, lcase.weights, outputs={"idx_attn": idx}, events=evs)
-    reps = 3
-    stage_ms = np.zeros(len(S.LAYER_STAGES))
+    # per-stage median of several staged passes (a single pass right after
+    # the timed loop can catch a clock transient)
+    reps = 9
+    per_rep = []
     for _ in range(reps):
         S.spts_layer_forward(hb, lcase.pos, ldesc, lcase.weights, events=evs)
         torch.cuda.synchronize()
-        stage_ms += np.array([evs[i].elapsed_time(evs[i + 1]) for i in range(len(S.LAYER_STAGES))])
-    stage_ms /= reps
+        per_rep.append([evs[i].elapsed_time(evs[i + 1]) for i in range(len(S.LAYER_STAGES))])
+    stage_ms = np.median(np.array(per_rep), axis=0)
     ffn = wl.F > 0
     fl, nbytes = layer_work(wl, wl.N, ldesc.k, wl.P, idx.cpu().numpy(), ffn)
     kernel_stages = ["k_proj_rope", "v_proj", "q_proj_rope", "reduced_attention", "o_proj_scatter", "ltp_scores",
