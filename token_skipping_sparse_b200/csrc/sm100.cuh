@@ -25,8 +25,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
-__device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 
 // Number of a[0..n) that are <= v (a sorted ascending), by the whole warp:
 // each step samples 32 evenly spaced points, so 2^17 keys take 4 dependent
