@@ -42,11 +42,14 @@ def test_linear_store_more_tiles_than_sm_pairs():
     assert_bf16_close(np64(out), want, 1e-4, "linear store, many tiles")
 
 
-def test_linear_rope():
+@pytest.mark.parametrize("lo,hi", [(0, 200000), (2 ** 24 - 170, 2 ** 24 + 163), (2 ** 30, 2 ** 31 - 1)])
+def test_linear_rope(lo, hi):
+    # positions below 2^24 take the fp32 two-product angle reduction, from
+    # 2^24 on the fp64 one; the middle case straddles the switch
     M, K, H = 333, 512, 4
     A = torch.randn(M, K).to(torch.bfloat16)
     W = _w(H * 128, K)
-    pos = torch.from_numpy(np.sort(rng.choice(200000, M, replace=False)).astype(np.int32))
+    pos = torch.from_numpy(np.sort(rng.choice(np.arange(lo, hi), M, replace=False)).astype(np.int32))
     out = S.spts_linear(A.cuda(), W.cuda(), S.EPI_ROPE, row_pos=pos.cuda(), theta=500000.0)
     want = O.bf16_round(O.rope((np64(A) @ np64(W).T).reshape(M, H, 128), pos.numpy(), 500000.0)).reshape(M, -1)
     assert_bf16_close(np64(out), want, 1e-4, "linear rope")
@@ -62,12 +65,16 @@ def test_linear_swiglu():
     assert_bf16_close(np64(out), want, 1e-4, "linear swiglu")
 
 
-def test_linear_scatter_add():
-    M, K, N, Nc = 200, 384, 512, 700
+@pytest.mark.parametrize("M,sort_rows", [(200, True), (200, False), (100, False), (1, True)])
+def test_linear_scatter_add(M, sort_rows):
+    # two-SM tiles (M > 128) and one-SM tiles, ragged last tiles, rows in any
+    # order (they must only be unique)
+    K, N, Nc = 384, 512, 700
     A = torch.randn(M, K).to(torch.bfloat16)
     W = _w(N, K)
     h = torch.randn(Nc, N)
-    rows = torch.from_numpy(np.sort(rng.choice(Nc, M, replace=False)).astype(np.int32))
+    rows = rng.choice(Nc, M, replace=False)
+    rows = torch.from_numpy((np.sort(rows) if sort_rows else rows).astype(np.int32))
     hd = h.cuda()
     S.spts_linear(A.cuda(), W.cuda(), S.EPI_SCATTER_ADD, out=hd, rows=rows.cuda())
     want = np64(h)
@@ -88,9 +95,10 @@ def test_rmsnorm_rows_with_gather():
     assert_bf16_close(np64(y), want, 1e-5, "rmsnorm")
 
 
-def test_rope_inplace():
+@pytest.mark.parametrize("lo,hi", [(0, 131072), (2 ** 24 - 45, 2 ** 24 + 45)])
+def test_rope_inplace(lo, hi):
     x = torch.randn(90, 8, 128).to(torch.bfloat16)
-    pos = torch.from_numpy(np.sort(rng.choice(131072, 90, replace=False)).astype(np.int32))
+    pos = torch.from_numpy(np.sort(rng.choice(np.arange(lo, hi), 90, replace=False)).astype(np.int32))
     y = S.spts_rope(x.cuda(), pos.cuda(), 500000.0)
     want = O.bf16_round(O.rope(np64(x), pos.numpy(), 500000.0))
     assert_bf16_close(np64(y), want, 1e-5, "rope")

@@ -33,7 +33,7 @@ __device__ __forceinline__ void rope_cos_sin(int32_t pos, const RopeFreqs &f, in
     const float lo = fmaf(pf, f.turn_hi[i], -hi);
     t = (hi - rintf(hi)) + (lo + pf * f.turn_lo[i]);
   } else {
-    const double a = static_cast<double>(pos) * (static_cast<double>(f.turn_hi[i]) + f.turn_lo[i]);
+    const double a = static_cast<double>(pos) * f.inv_freq[i] * 0.15915494309189533576888376337251;
     t = static_cast<float>(a - rint(a));
   }
   __sincosf(t * 6.28318530717958647692f, s, c);
