@@ -163,6 +163,9 @@ def test_fuse_modes_exact_values():
     c = np.array([8, 4, 2, 1], np.float32)
     f = O.fuse_scores(s, c, O.FUSE_MAXNORM_ADD, 0.5, 0.5)
     np.testing.assert_array_equal(f, np.array([0.5625, 0.375, 0.375, 0.5625], np.float32))
+    # unequal weights: 0.25 s/8 + 0.75 c/8, exact in fp32
+    f = O.fuse_scores(s, c, O.FUSE_MAXNORM_ADD, 0.25, 0.75)
+    np.testing.assert_array_equal(f, np.array([0.78125, 0.4375, 0.3125, 0.34375], np.float32))
     f = O.fuse_scores(s, c, O.FUSE_MULTIPLY)
     np.testing.assert_array_equal(f, (torch.from_numpy(s) * torch.from_numpy(c)).numpy())
     np.testing.assert_array_equal(O.fuse_scores(s, c, O.FUSE_NONE), s)
@@ -387,6 +390,37 @@ def test_layer_skipped_rows_pass_through():
     assert np.array_equal(out[skip], h[skip])
     assert set(range(60, 64)) <= set(tr["idx_attn"]) and set(range(60, 64)) <= set(tr["idx_ffn"])
     assert len(tr["idx_attn"]) == 20 and np.all(np.diff(tr["idx_attn"]) > 0)
+
+
+def _top_k_rows(score, k, tail):
+    """Top-k by plain sorting (largest first, ties to the lower index), the
+    last `tail` rows forced, ascending."""
+    n = len(score)
+    free = sorted(range(n - tail), key=lambda i: (-float(score[i]), i))[: k - tail]
+    return np.array(sorted(free) + list(range(n - tail, n)))
+
+
+@pytest.mark.parametrize("w_a,w_b", [(0.0, 1.0), (1.0, 0.0)])
+def test_layer_selection_wiring(w_a, w_b):
+    # with one fusion weight zero, the FFN rows are the top-k of one score:
+    # of the LTP score of RMSNorm(h') (h' = the attention output) for w_a =
+    # 0, of the probe score for w_b = 0 (the attention rows); attention
+    # changes exactly its rows of h, the FFN exactly its rows of h'
+    h, pos, W, cfg = _tiny_layer(N=40, k=12, P=3)
+    cfg.w_a, cfg.w_b = w_a, w_b
+    tr = {}
+    out, _ = O.layer_forward(h, pos, W, cfg, tr)
+    # the probes are the last P rows, at their own positions
+    Hq, d = cfg.Hq, cfg.d
+    q_probe = O.bf16_round(O.rope((tr["xn"][-3:] @ W.w_q.T).reshape(3, Hq, d), pos[-3:]))
+    np.testing.assert_allclose(tr["s"], O.probe_scores(q_probe, pos[-3:], tr["k"], pos)[0], rtol=1e-12)
+    want_a = _top_k_rows(tr["s"].astype(np.float32), 12, 3)
+    assert np.array_equal(tr["idx_attn"], want_a)
+    assert np.array_equal(np.nonzero(np.any(tr["h_attn"] != h, axis=1))[0], want_a)
+    c = O.ltp_scores(O.bf16_round(O.rmsnorm(tr["h_attn"], W.norm_ffn, cfg.eps)), W.ltp_a, W.ltp_b)
+    want_f = _top_k_rows(c.astype(np.float32), 12, 3) if w_a == 0 else want_a
+    assert np.array_equal(tr["idx_ffn"], want_f)
+    assert np.array_equal(np.nonzero(np.any(out != tr["h_attn"], axis=1))[0], want_f)
 
 
 def test_msdp_all_ratios_one_is_dense_stack_and_sets_nest():
