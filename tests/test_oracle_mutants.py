@@ -18,7 +18,7 @@ import tests.test_oracle_pins as PINS
 
 _ORIG = {n: getattr(OS, n) for n in ("rmsnorm", "rope", "probe_scores", "ltp_scores", "ltp_topm_scores",
                                      "fuse_scores", "select_topk", "reduced_attention", "attention_residual",
-                                     "reduced_ffn", "inject_salience")}
+                                     "reduced_ffn", "inject_salience", "stage_prune")}
 
 
 # ---------------------------------------------------------------- mutants
@@ -163,18 +163,27 @@ def _salience_not_unit(kk, q_probe, rows, shift, Hkv):
     return kk
 
 
-def _layer_with(old, new):
-    """The oracle's composed layer with one line of its source changed."""
+def _stage_prune_lowest(scores, k_keep, force_tail, h, pos):
+    return _ORIG["stage_prune"](-np.asarray(scores, dtype=np.float32), k_keep, force_tail, h, pos)
+
+
+def _source_with(fn, old, new):
+    """An oracle function with one line of its source changed."""
     import inspect
     import textwrap
-    src = textwrap.dedent(inspect.getsource(_ORIG_LAYER))
+    src = textwrap.dedent(inspect.getsource(fn))
     assert src.count(old) == 1, old
     ns = dict(vars(OS))
     exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)  # noqa: S102
-    return ns["layer_forward"]
+    return ns[fn.__name__]
 
 
 _ORIG_LAYER = OS.layer_forward
+_ORIG_MSDP = OS.msdp_forward
+
+
+def _layer_with(old, new):
+    return _source_with(_ORIG_LAYER, old, new)
 _LAYER_PINS = ["test_layer_keep_all_equals_dense_layer", "test_layer_skipped_rows_pass_through",
                ("test_layer_selection_wiring", (0.0, 1.0)), ("test_layer_selection_wiring", (1.0, 0.0))]
 
@@ -227,6 +236,15 @@ MUTANTS = {
         "layer_forward", _layer_with("pp = pos[Nc - P:]", "pp = pos[:P]"), _LAYER_PINS),
     "FFN built on the pre-attention stream": (
         "layer_forward", _layer_with("h2 = reduced_ffn(h1,", "h2 = reduced_ffn(h,"), _LAYER_PINS),
+    "stage prune keeps the lowest scores": ("stage_prune", _stage_prune_lowest,
+                                            ["test_stage_prune_worked_example",
+                                             "test_msdp_prunes_by_the_last_layers_fused_score"]),
+    "MSDP prunes by the stage's first layer": (
+        "msdp_forward",
+        _source_with(OS.msdp_forward, "            h, f = layer_forward(h, pos, layers[li], cfg, tr)",
+                     "            h, f_l = layer_forward(h, pos, layers[li], cfg, tr)\n"
+                     "            f = f_l if f is None else f"),
+        ["test_msdp_prunes_by_the_last_layers_fused_score", "test_msdp_all_ratios_one_is_dense_stack_and_sets_nest"]),
     "salience direction not normalised": ("inject_salience", _salience_not_unit, ["test_inject_salience_closed_form"]),
 }
 

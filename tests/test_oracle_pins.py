@@ -448,6 +448,35 @@ def test_msdp_all_ratios_one_is_dense_stack_and_sets_nest():
     assert set(opos.tolist()) == seen and {pos[-1], pos[-2]} <= seen
 
 
+def test_msdp_prunes_by_the_last_layers_fused_score():
+    # at each stage boundary the candidates kept are the top-k_s of the
+    # stage's last layer's fused score (plain sorting, tail forced)
+    h, pos, W0, cfg = _tiny_layer(N=40, P=2)
+    layers = [_tiny_layer(N=40, P=2)[2] for _ in range(6)]
+    m = O.MsdpConfig(layer=cfg, ratios=("0.75", "0.5", "0.3"), layers_per_stage=2)
+    tr = []
+    out, opos, pruned = O.msdp_forward(h, pos, layers, m, tr)
+    cand = pos
+    for s_i, r in enumerate(m.ratios):
+        k_s = O.keep_count(r, 40)
+        last = tr[2 * s_i + 1]
+        keep = _top_k_rows(last["f"], k_s, 2)
+        nxt = cand[keep]
+        assert np.array_equal(np.sort(pruned[s_i][0]), np.setdiff1d(cand, nxt))
+        cand = nxt
+    assert np.array_equal(opos, cand)
+
+
+def test_stage_prune_worked_example():
+    scores = np.array([0.1, 0.9, 0.5, 0.9, 0.3, 0.2], np.float32)
+    h = np.arange(12.0).reshape(6, 2)
+    pos = np.array([3, 8, 9, 20, 21, 30])
+    # keep 4, tail 1: the top 3 of the first 5 (0.9 at 1 and 3, then 0.5 at 2), then row 5
+    ho, po, kept = O.stage_prune(scores, 4, 1, h, pos)
+    assert list(kept) == [1, 2, 3, 5] and list(po) == [8, 9, 20, 30]
+    np.testing.assert_array_equal(ho, h[[1, 2, 3, 5]])
+
+
 def test_schedule_without_skipping_is_the_dense_stack_and_sets_nest():
     # budgets and the final count at least N: every layer is a full layer
     h, pos, W0, cfg = _tiny_layer(N=40, P=2)
