@@ -70,6 +70,27 @@ def test_attention_single_partial_tile_and_first_position():
     assert_bf16_close(np64(o)[0], v0, 1e-6, "first-position query")
 
 
+@pytest.mark.parametrize("n_blind", [3, 70])
+def test_attention_queries_that_see_no_key_are_zero(n_blind):
+    # keys start at position 1000; the first n_blind queries sit before them
+    # (3: inside the first Q tile, 70: whole tiles of them), the rest among
+    # the keys: the blind rows come out 0, the others match the oracle
+    Nc, Hq, Hkv = 400, 8, 2
+    pos = (1000 + np.sort(rng.choice(4000, Nc, replace=False))).astype(np.int32)
+    blind = np.sort(rng.choice(1000, n_blind, replace=False)).astype(np.int32)
+    seen = np.sort(rng.choice(pos, 90, replace=False)).astype(np.int32)
+    q_pos = np.concatenate([blind, seen])
+    m = len(q_pos)
+    q = torch.randn(m, Hq, 128).to(torch.bfloat16)
+    kk = torch.randn(Nc, Hkv, 128).to(torch.bfloat16)
+    v = torch.randn(Nc, Hkv, 128).to(torch.bfloat16)
+    o = np64(S.spts_reduced_attention(q.cuda(), torch.from_numpy(q_pos).cuda(), kk.cuda(), v.cuda(),
+                                      torch.from_numpy(pos).cuda()))
+    assert np.array_equal(o[:n_blind], np.zeros_like(o[:n_blind]))
+    want = O.reduced_attention(np64(q)[n_blind:], seen, np64(kk), np64(v), pos)
+    assert_close(o[n_blind:], want, 2e-2, "attention after the blind rows")
+
+
 def test_probe_single_probe_and_all_keys_are_probes():
     for Nc, P in [(777, 1), (64, 64)]:
         pos = np.sort(rng.choice(5000, Nc, replace=False)).astype(np.int32)
