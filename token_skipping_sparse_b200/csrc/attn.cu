@@ -11,10 +11,13 @@
 //               find the tiles' key ranges by warp-wide searches), then the
 //               other K and V tiles of 128 keys into a 2-stage ring
 //               (128-byte swizzle);
-//   warp 1      MMA, per key tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).
+//   warp 1      MMA, per key tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1),
+//               the whole warp running the loop on warp-uniform descriptors
+//               and one elected lane issuing each tcgen05 op (a lone lane
+//               under a lane test issued them markedly slower);
 //               S_X = Q_X K^T lands in TMEM region S_X; the softmax writes
 //               bf16 P over it and PV reads P from TMEM (A operand in TMEM)
-//               with V an MN-major shared-memory operand, into O_X.
+//               with V an MN-major shared-memory operand, into O_X;
 //   warps 2..3  idle (they complete warpgroup 0 for the register split);
 //   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B, one thread
 //               per Q row: tcgen05.ld of the S row, causal mask (only on key
@@ -201,17 +204,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
-    if (lane == 0) {
+    {  // the whole warp runs the issue loop; one elected lane issues each MMA and commit
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, BKV, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status, p.wait_ns, 0x22u);
+      auto wait_all = [&](uint64_t *bar, uint32_t parity, uint32_t where) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status, p.wait_ns, where));
+      };
+      bool ok = wait_all(q_full, 0, 0x22u);
       tc_fence_after();
       // S_X(j) into TMEM region S_X.  tcgen05.mma from this thread run in
       // issue order, so S_X(j+1) (issued after PV_X(j)) cannot overwrite P_X(j)
       // before PV_X(j) has read it.
       auto issue_s = [&](int x, int j) -> bool {
         const int st = j % KV_STAGES;
-        if (!mbar_wait(&k_full[st], (j / KV_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x23u)) return false;
+        if (!wait_all(&k_full[st], (j / KV_STAGES) & 1, 0x23u)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(sK + st * TILE_BYTES);
         const uint32_t q_addr = smem_u32(sQ + x * TILE_BYTES);
@@ -219,23 +225,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t a = sdesc_k_sw128(q_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3);
           const uint64_t b = sdesc_k_sw128(k_addr + (kk >> 2) * CHUNK_BYTES) + 2 * (kk & 3);
-          mma_bf16_ss(tmem + x * BKV, a, b, idesc_s, kk > 0);
+          mma_bf16_ss_w(tmem + x * BKV, a, b, idesc_s, kk > 0);
         }
-        tc_commit(&s_full[x]);
+        tc_commit_w(&s_full[x]);
         return true;
       };
       auto issue_pv = [&](int x, int j) -> bool {
         const int st = j % KV_STAGES;
-        if (!mbar_wait(&p_ready[x], j & 1, abort_flag, p.status, p.wait_ns, 0x24u)) return false;
-        if (!mbar_wait(&v_full[st], (j / KV_STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x25u)) return false;
+        if (!wait_all(&p_ready[x], j & 1, 0x24u)) return false;
+        if (!wait_all(&v_full[st], (j / KV_STAGES) & 1, 0x25u)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(sV + st * TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t v = sdesc_mn_sw128(v_addr + kk * 16 * 128, CHUNK_BYTES);
-          mma_bf16_ts(tmem + 256 + x * 128, tmem + x * BKV + kk * 8, v, idesc_pv, (j | kk) != 0);
+          mma_bf16_ts_w(tmem + 256 + x * 128, tmem + x * BKV + kk * 8, v, idesc_pv, (j | kk) != 0);
         }
-        tc_commit(&o_done[x]);
+        tc_commit_w(&o_done[x]);
         return true;
       };
       for (int x = 0; ok && x < 2; ++x)
@@ -247,9 +253,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           ok = issue_pv(x, j);
           if (ok && j + 1 < nxx) ok = issue_s(x, j + 1);
         }
-        if (ok) tc_commit(&kv_empty[j % KV_STAGES]);  // both tiles are done with K/V tile j
+        if (ok) tc_commit_w(&kv_empty[j % KV_STAGES]);  // both tiles are done with K/V tile j
       }
-      tc_commit(drain);
+      tc_commit_w(drain);
       mbar_drain(drain, 0, p.status);
     }
     __syncwarp();
