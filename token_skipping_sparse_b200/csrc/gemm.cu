@@ -9,8 +9,9 @@
 // larger M uses the two-SM 256 x 256 tiles further down):
 //   warp 0      TMA producer: A tile 128x64 and B tile 256x64 per stage into
 //               a 4-stage ring of 128-byte-swizzled shared memory;
-//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
-//               K=16) into one of two TMEM accumulators (2 x 256 columns);
+//   warp 1      MMA issuer: the warp runs the loop, one elected lane
+//               issues tcgen05.mma (M=128, N=256, K=16) into one of two TMEM
+//               accumulators (2 x 256 columns);
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (warp w reads
 //               TMEM lanes 32*(w%4)..+31), then the fused epilogue and the
 //               global stores, overlapping the next tile's main loop.
@@ -252,7 +253,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // the whole warp runs the issue loop; one elected lane issues each MMA and commit
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
       int stage = 0;
       uint32_t phase = 0;
@@ -261,11 +262,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, p.wait_ns, 0x12u)) break;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, p.wait_ns, 0x12u)))
+          break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, p.wait_ns, 0x13u)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, p.status, p.wait_ns, 0x13u))) {
             ok = false;
             break;
           }
@@ -274,17 +277,17 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint64_t bdesc = sdesc_k_sw128(smem_u32(sB + stage * B_BYTES));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
-          tc_commit(&empty[stage]);
+            mma_bf16_ss_w(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+          tc_commit_w(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (ok) tc_commit(&tfull[acc]);
+        if (ok) tc_commit_w(&tfull[acc]);
       }
       // every MMA issued so far must finish before TMEM is released
-      tc_commit(drain);
+      tc_commit_w(drain);
       mbar_drain(drain, 0, p.status);
     }
     __syncwarp();
@@ -341,8 +344,9 @@ spts_status launch_epi(const GemmArgs &g, const CUtensorMap &ta, const CUtensorM
 // 4 KB of A and 8 KB of B.
 //   warp 0      TMA in both CTAs; every copy completes on CTA 0's full[]
 //               barrier, whose expected bytes CTA 0 posts for both halves;
-//   warp 1      CTA 0: MMA issuer for the pair (stage and accumulator
-//               releases are commits multicast to both CTAs);
+//   warp 1      CTA 0: MMA issuer for the pair, warp-wide with one elected
+//               lane issuing (stage and accumulator releases are commits
+//               multicast to both CTAs);
 //   warps 2..5  epilogue of this CTA's rows; they release an accumulator on
 //               CTA 0's tempty[] barrier (128 arrivals from each CTA).
 // Loads are plain tile loads (no multicast): each CTA reads only its own
@@ -437,7 +441,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
+    if (rank == 0) {  // the whole warp runs the issue loop; one elected lane issues each MMA and commit
       constexpr uint32_t idesc = idesc_bf16_f32(256, BN, 0, 0);
       int stage = 0;
       uint32_t phase = 0;
@@ -446,11 +450,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int t = pair; t < tiles && ok; t += n_pairs, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
-        if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, p.wait_ns, 0x32u)) break;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, p.wait_ns, 0x32u)))
+          break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, p.wait_ns, 0x33u)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, p.status, p.wait_ns, 0x33u))) {
             ok = false;
             break;
           }
@@ -459,17 +465,17 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint64_t bdesc = sdesc_k_sw128(smem_u32(sB + stage * HALF_BYTES));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma2_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
-          tc2_commit_both(&empty[stage]);
+            mma2_bf16_ss_w(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+          tc2_commit_both_w(&empty[stage]);
           if (++stage == STAGES2) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (ok) tc2_commit_both(&tfull[acc]);
+        if (ok) tc2_commit_both_w(&tfull[acc]);
       }
       // every MMA issued so far (they write both CTAs' TMEM) must finish
-      tc2_commit_self(drain);
+      tc2_commit_self_w(drain);
       mbar_drain(drain, 0, p.status);
     }
     __syncwarp();
