@@ -345,9 +345,13 @@ typedef struct {
   int32_t *idx_ffn;    /* [k] rows that ran the reduced FFN      */
   void *o_sel;         /* [k, Hq, d] bf16 reduced-attention out  */
   float *h_attn;       /* [Nc, D] residual after attention       */
-  /* NULL, or SPTS_LAYER_STAGE_EVENTS cudaEvent_t handles created by the
-   * caller; event i is recorded on the stream after stage i (see below),
-   * event 0 before the first kernel.  A measurement aid. */
+  /* NULL, or an array of SPTS_LAYER_STAGE_EVENTS cudaEvent_t handles
+   * created by the caller, any of which may be NULL (not recorded); event i
+   * is recorded on the stream after stage i (see below), event 0 before the
+   * first kernel.  When any of events 1..7 is given, every kernel runs on
+   * the caller's stream so that stage times add up; otherwise the probe-Q
+   * and V projections still run on the library's side stream (event 8
+   * follows the join with it).  A measurement aid. */
   void *const *stage_events;
 } spts_layer_outputs;
 

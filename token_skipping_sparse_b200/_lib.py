@@ -385,14 +385,15 @@ def stage_events():
 
 def spts_layer_forward(h, pos, desc, weights, outputs=False, ws=None, events=None):
     """Runs one layer in place on h [Nc, D] fp32; returns a dict of the
-    optional outputs when outputs=True.  `events` (from stage_events()) are
-    recorded at the stage boundaries."""
+    optional outputs when outputs=True.  `events` (from stage_events(), or a
+    list of LAYER_STAGE_EVENTS entries some of which are None) are recorded
+    at the stage boundaries."""
     Nc = h.shape[0]
     out = None
     res = {}
     ev_arr = None
     if events is not None:
-        ev_arr = (C.c_void_p * LAYER_STAGE_EVENTS)(*[e.cuda_event for e in events])
+        ev_arr = (C.c_void_p * LAYER_STAGE_EVENTS)(*[e.cuda_event if e is not None else None for e in events])
     if outputs is not False or events is not None:
         out = LayerOutputs()
         out.stage_events = C.cast(ev_arr, C.c_void_p) if ev_arr is not None else None

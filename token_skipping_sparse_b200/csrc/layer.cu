@@ -109,7 +109,8 @@ spts_status dense_layer(const spts_layer_desc *L, const spts_layer_weights *W, f
   const float scale = 1.0f / sqrtf(static_cast<float>(L->d));
   void *osel = o.o_sel ? o.o_sel : b.osel;
   auto mark = [&](int i) -> spts_status {
-    if (o.stage_events != nullptr) SPTS_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(o.stage_events[i]), s));
+    if (o.stage_events != nullptr && o.stage_events[i] != nullptr)
+      SPTS_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(o.stage_events[i]), s));
     return SPTS_OK;
   };
   SPTS_TRY(mark(0));
@@ -180,16 +181,19 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   void *osel = o.o_sel ? o.o_sel : b.osel;
   const float scale = 1.0f / sqrtf(static_cast<float>(L->d));
   auto mark = [&](int i) -> spts_status {
-    if (o.stage_events != nullptr) {
+    if (o.stage_events != nullptr && o.stage_events[i] != nullptr)
       SPTS_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(o.stage_events[i]), s));
-    }
     return SPTS_OK;
   };
 
-  // Stage events time the stages one after another, so with them the side
-  // stream is not used and every kernel runs on the caller's stream.
+  // Events 1..7 time stages that overlap the side stream's projections: when
+  // any of them is requested every kernel runs on the caller's stream, so
+  // the stage times add up.  Event 0 and events 8.. leave the side stream on.
+  bool serial = false;
+  if (o.stage_events != nullptr)
+    for (int i = 1; i <= 7; ++i) serial = serial || o.stage_events[i] != nullptr;
   SideStream *side = nullptr;
-  if (o.stage_events == nullptr) SPTS_TRY(side_stream(&side));
+  if (!serial) SPTS_TRY(side_stream(&side));
   // On any early return after the fork, still order the caller's stream
   // behind the side stream's work on the workspace.
   struct JoinGuard {
@@ -244,11 +248,11 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   SPTS_TRY(mark(7));
   GemmArgs gqs{b.xsel, k, D, W->w_q, nullptr, hq, SPTS_EPI_ROPE, b.qsel, nullptr, b.qpos, L->theta, st};
   SPTS_TRY(launch_gemm(gqs, s));
-  SPTS_TRY(mark(8));
   if (side) {  // join: V is ready
     SPTS_CUDA_TRY(cudaStreamWaitEvent(s, side->v_done, 0));
     guard.joined = true;
   }
+  SPTS_TRY(mark(8));
   if (kv_active) {
     // keys and values of the active rows only: K gathered, V projected from
     // the gathered normalised rows, key positions = the active positions

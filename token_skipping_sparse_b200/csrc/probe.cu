@@ -165,22 +165,26 @@ __device__ __forceinline__ void producer(const Smem &s, const Geo &p, const CUte
   }
 }
 
-// warp 1: for each key tile, one 8-MMA group per sub-item into its buffer.
+// warp 1 (the whole warp; one elected lane issues each MMA and commit): for
+// each key tile, one 8-MMA group per sub-item into its buffer.
 // Pass 1: D = Q_u K^T (A = row tile u, B = K tile).  Pass 2: D = K Q_u^T
 // (A = K tile, B = column chunk u of the probe rows).
 __device__ __forceinline__ void mma_issuer(const Smem &s, const Geo &p, uint32_t tmem, int n, bool transposed) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
-  bool ok = mbar_wait(s.q_full, 0, s.abort_flag, p.status, p.wait_ns, 0x32u);
+  bool ok = __all_sync(0xffffffffu, mbar_wait(s.q_full, 0, s.abort_flag, p.status, p.wait_ns, 0x32u));
   tc_fence_after();
   const uint32_t q_addr = smem_u32(s.q);
   for (int i = 0; ok && i < n; ++i) {
     const int st = i % p.stages;
-    if (!mbar_wait(&s.k_full[st], (i / p.stages) & 1, s.abort_flag, p.status, p.wait_ns, 0x33u)) break;
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait(&s.k_full[st], (i / p.stages) & 1, s.abort_flag, p.status, p.wait_ns, 0x33u)))
+      break;
     const uint32_t k_addr = smem_u32(s.k + st * TILE_BYTES);
     for (int u = 0; ok && u < p.n_sub; ++u) {
       const int b = (i & 1) * 2 + (u & 1);
       const uint32_t use = buffer_uses(i, u, p.n_sub);
-      if (!mbar_wait(&s.s_free[b], (use & 1u) ^ 1u, s.abort_flag, p.status, p.wait_ns, 0x34u)) {
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&s.s_free[b], (use & 1u) ^ 1u, s.abort_flag, p.status, p.wait_ns, 0x34u))) {
         ok = false;
         break;
       }
@@ -191,13 +195,13 @@ __device__ __forceinline__ void mma_issuer(const Smem &s, const Geo &p, uint32_t
         const uint32_t qc = transposed ? q_addr + ((kk >> 2) * p.n_sub + u) * CHUNK_BYTES
                                        : q_addr + u * TILE_BYTES + (kk >> 2) * CHUNK_BYTES;
         const uint64_t qd = sdesc_k_sw128(qc) + 2 * (kk & 3), kd = sdesc_k_sw128(kc) + 2 * (kk & 3);
-        mma_bf16_ss(tmem + b * 128, transposed ? kd : qd, transposed ? qd : kd, idesc, kk > 0);
+        mma_bf16_ss_w(tmem + b * 128, transposed ? kd : qd, transposed ? qd : kd, idesc, kk > 0);
       }
-      tc_commit(&s.s_full[b]);
+      tc_commit_w(&s.s_full[b]);
     }
-    if (ok) tc_commit(&s.k_empty[st]);
+    if (ok) tc_commit_w(&s.k_empty[st]);
   }
-  tc_commit(s.drain);
+  tc_commit_w(s.drain);
   mbar_drain(s.drain, 0, p.status);
 }
 
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
-    if (lane == 0) mma_issuer(s, p, tmem, n, false);
+    mma_issuer(s, p, tmem, n, false);
     __syncwarp();
   } else if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));  // idle
@@ -403,7 +407,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
-    if (lane == 0) mma_issuer(s, p, tmem, n, true);
+    mma_issuer(s, p, tmem, n, true);
     __syncwarp();
   } else if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));  // idle
