@@ -1,0 +1,68 @@
+"""Host-side pieces of bench.py checked on CPU: the algorithmic work it
+divides by (brute-force pair counts), and the ncu traffic figure it reports
+only while the captured kernel source is unchanged."""
+
+import os
+import shutil
+import types
+
+import numpy as np
+
+import bench
+
+
+def _wl(kv_active=False):
+    return types.SimpleNamespace(D=64, Hq=4, Hkv=2, d=16, F=96, r=8, ltp_dout=0, kv_active=kv_active)
+
+
+def _visible_pairs(q_rows, key_rows, pos):
+    # causal by original position: query row i sees key row j iff pos[j] <= pos[i]
+    return sum(1 for i in q_rows for j in key_rows if pos[j] <= pos[i])
+
+
+def test_attention_and_probe_flops_are_the_visible_pair_counts():
+    rng = np.random.default_rng(3)
+    Nc, k, P = 57, 13, 5
+    pos = np.sort(rng.choice(10 * Nc, Nc, replace=False))
+    idx = np.sort(rng.choice(Nc, k, replace=False))
+    wl = _wl()
+    fl, _ = bench.layer_work(wl, Nc, k, P, idx)
+    assert fl["reduced_attention"] == 4.0 * wl.Hq * wl.d * _visible_pairs(idx, range(Nc), pos)
+    probe_rows = range(Nc - P, Nc)
+    assert fl["probe_scores"] == 2.0 * 2.0 * wl.Hq * wl.d * _visible_pairs(probe_rows, range(Nc), pos)
+    # active-row keys: the selected queries attend to the selected keys only
+    wl_kv = _wl(kv_active=True)
+    fl_kv, _ = bench.layer_work(wl_kv, Nc, k, P, idx)
+    assert fl_kv["reduced_attention"] == 4.0 * wl.Hq * wl.d * _visible_pairs(idx, idx, pos)
+    assert fl_kv["v_proj"] == 2.0 * k * wl.D * wl.Hkv * wl.d
+
+
+def test_gemm_flops():
+    wl = _wl()
+    Nc, k, P = 40, 9, 3
+    fl, _ = bench.layer_work(wl, Nc, k, P, np.arange(k))
+    assert fl["gate_up_swiglu"] == 2 * (2.0 * k * wl.D * wl.F)
+    assert fl["down_proj_scatter"] == 2.0 * k * wl.F * wl.D
+    assert fl["q_proj_rope"] == 2.0 * k * wl.D * wl.Hq * wl.d
+    assert fl["ltp_scores"] == 2.0 * Nc * (wl.D * wl.r + wl.r * wl.D)
+
+
+def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch):
+    root = bench.ROOT
+    summary = os.path.join(root, "profiles", "attention_bf16_layer_32k.md")
+    if not os.path.exists(summary):
+        return
+    got = bench.captured_traffic("layer_32k")
+    assert got is not None and got > 0
+    assert bench.captured_traffic("no_such_workload") is None
+    # a copy of the tree whose kernel source differs by one byte: no figure
+    (tmp_path / "profiles").mkdir()
+    shutil.copy(summary, tmp_path / "profiles" / "attention_bf16_layer_32k.md")
+    src_dir = tmp_path / "token_skipping_sparse_b200" / "csrc"
+    src_dir.mkdir(parents=True)
+    text = open(os.path.join(root, "token_skipping_sparse_b200", "csrc", "attn.cu")).read()
+    (src_dir / "attn.cu").write_text(text + "\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.captured_traffic("layer_32k") is None
+    (src_dir / "attn.cu").write_text(text)
+    assert bench.captured_traffic("layer_32k") == got
