@@ -339,7 +339,8 @@ __device__ __forceinline__ void tc2_commit_self(uint64_t *bar) {
                : "memory");
 }
 
-// Warp-wide forms of the two above (one elected lane issues).
+// Warp-wide forms of mma2_bf16_ss, tc2_commit_both and tc2_commit_self: the
+// whole warp calls them converged, one elected lane issues.
 __device__ __forceinline__ void mma2_bf16_ss_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                                uint32_t accumulate) {
   asm volatile(
@@ -355,8 +356,7 @@ __device__ __forceinline__ void tc2_commit_both_w(uint64_t *bar) {
       "{\n\t.reg .pred e;\n\t"
       "elect.sync _|e, 0xffffffff;\n\t"
       "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-      "\n\t}\n" ::"r"(
-          smem_u32(bar)),
+      "\n\t}\n" ::"r"(smem_u32(bar)),
       "h"(static_cast<uint16_t>(3))
       : "memory");
 }
