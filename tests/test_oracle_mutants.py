@@ -17,8 +17,8 @@ import oracle.spts as OS
 import tests.test_oracle_pins as PINS
 
 _ORIG = {n: getattr(OS, n) for n in ("rmsnorm", "rope", "probe_scores", "ltp_scores", "ltp_topm_scores",
-                                     "fuse_scores", "select_topk", "reduced_attention", "attention_residual",
-                                     "reduced_ffn", "inject_salience", "stage_prune")}
+                                     "fuse_scores", "select_topk", "select_sequential", "reduced_attention",
+                                     "attention_residual", "reduced_ffn", "inject_salience", "stage_prune")}
 
 
 # ---------------------------------------------------------------- mutants
@@ -163,6 +163,15 @@ def _salience_not_unit(kk, q_probe, rows, shift, Hkv):
     return kk
 
 
+def _sequential_scores_swapped(s, c, k_pool, k, force_tail):   # pool by c, decided by s
+    return _ORIG["select_sequential"](c, s, k_pool, k, force_tail)
+
+
+def _sequential_pool_local(s, c, k_pool, k, force_tail):   # indices into the pool, not the candidates
+    pool, _ = _ORIG["select_topk"](np.asarray(s, dtype=np.float32), k_pool, force_tail)
+    return _ORIG["select_topk"](np.asarray(c, dtype=np.float32)[pool], k, force_tail)
+
+
 def _stage_prune_lowest(scores, k_keep, force_tail, h, pos):
     return _ORIG["stage_prune"](-np.asarray(scores, dtype=np.float32), k_keep, force_tail, h, pos)
 
@@ -180,6 +189,7 @@ def _source_with(fn, old, new):
 
 _ORIG_LAYER = OS.layer_forward
 _ORIG_MSDP = OS.msdp_forward
+_ORIG_SCHEDULE = OS.schedule_forward
 
 
 def _layer_with(old, new):
@@ -246,6 +256,31 @@ MUTANTS = {
                      "            f = f_l if f is None else f"),
         ["test_msdp_prunes_by_the_last_layers_fused_score", "test_msdp_all_ratios_one_is_dense_stack_and_sets_nest"]),
     "salience direction not normalised": ("inject_salience", _salience_not_unit, ["test_inject_salience_closed_form"]),
+    "sequential select with the scores swapped": (
+        "select_sequential", _sequential_scores_swapped,
+        [("test_select_sequential_reductions", (60,)), ("test_select_sequential_reductions", (20,))]),
+    "sequential select returns pool positions": (
+        "select_sequential", _sequential_pool_local,
+        [("test_select_sequential_reductions", (33,)), ("test_select_sequential_reductions", (60,))]),
+    "schedule prunes to the next stage's budget": (
+        "schedule_forward",
+        _source_with(_ORIG_SCHEDULE,
+                     "k_next = min(budgets[stage] if stage + 1 < len(stage_ends) else after_last, Nc)",
+                     "k_next = min(budgets[stage + 1] if stage + 1 < len(stage_ends) else after_last, Nc)"),
+        ["test_schedule_without_skipping_is_the_dense_stack_and_sets_nest"]),
+    "schedule prunes without keeping the probe tail": (
+        "schedule_forward",
+        _source_with(_ORIG_SCHEDULE, "kept, _ = select_topk(f, k_next, cfg.P)", "kept, _ = select_topk(f, k_next, 0)"),
+        ["test_schedule_without_skipping_is_the_dense_stack_and_sets_nest"]),
+    "schedule skips before the first skipping layer": (
+        "schedule_forward",
+        _source_with(_ORIG_SCHEDULE, "skip = l >= first_skip and", "skip = l >= 0 and"),
+        ["test_schedule_without_skipping_is_the_dense_stack_and_sets_nest"]),
+    "schedule keeps skipping after the last stage": (
+        "schedule_forward",
+        _source_with(_ORIG_SCHEDULE, "k = min(budgets[stage], Nc) if skip else Nc",
+                     "k = min(budgets[min(stage, len(budgets) - 1)], Nc) if l >= first_skip else Nc"),
+        ["test_schedule_without_skipping_is_the_dense_stack_and_sets_nest"]),
 }
 
 

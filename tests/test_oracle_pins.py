@@ -498,6 +498,13 @@ def test_schedule_without_skipping_is_the_dense_stack_and_sets_nest():
     for a, b in zip(tr, tr[1:]):
         assert set(b["cand"]) <= set(a["cand"])
     assert np.array_equal(opos, tr[-1]["cand"]) and out.shape == (10, h.shape[1])
+    # more survivors than the last stage's budget: the layers after the last
+    # stage are still full layers over every survivor
+    tr = []
+    out, opos = O.schedule_forward(h, pos, layers, cfg, 1, (2, 4), (30, 20), 25, tr)
+    assert [t["k"] for t in tr] == [40, 30, 30, 20, 20, 25]
+    assert [len(t["cand"]) for t in tr] == [40, 40, 40, 30, 30, 25]
+    assert not tr[-1]["skip"] and np.array_equal(np.sort(tr[-1]["sel_pos"]), np.sort(tr[-1]["cand"]))
 
 
 # ---------------------------------------------------------------- synthetic salience
