@@ -68,6 +68,22 @@ def _probe_unscaled(q_probe, probe_pos, k, key_pos, scale=None):
     return _ORIG["probe_scores"](q_probe, probe_pos, k, key_pos, 1.0)
 
 
+def _probe_mask_after_softmax(q_probe, probe_pos, k, key_pos, scale=None):
+    # each row normalised over every key, the future keys zeroed afterwards
+    q_probe, k = np.asarray(q_probe, dtype=np.float64), np.asarray(k, dtype=np.float64)
+    P, Hq, d = q_probe.shape
+    Nc, Hkv, _ = k.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    visible = np.asarray(key_pos)[None, :] <= np.asarray(probe_pos)[:, None]
+    group = np.zeros((Hkv, Nc))
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        logits = scale * (q_probe[:, h, :] @ k[:, g, :].T)
+        e = np.exp(logits - logits.max(axis=1, keepdims=True))
+        group[g] += np.where(visible, e / e.sum(axis=1, keepdims=True), 0.0).sum(axis=0)
+    return group.sum(axis=0), group
+
+
 def _ltp_squared(x, A, B):
     return _ORIG["ltp_scores"](x, A, B) ** 2
 
@@ -198,6 +214,8 @@ _LAYER_PINS = ["test_layer_keep_all_equals_dense_layer", "test_layer_skipped_row
                ("test_layer_selection_wiring", (0.0, 1.0)), ("test_layer_selection_wiring", (1.0, 0.0))]
 
 
+_ORIG_PROBE = OS.probe_scores
+
 # name -> (oracle function, mutant, pins that cover it)
 MUTANTS = {
     "rmsnorm over the wrong axis": ("rmsnorm", _rmsnorm_wrong_axis, ["test_rmsnorm_matches_torch"]),
@@ -215,6 +233,13 @@ MUTANTS = {
                                        "test_probe_scores_invariants_and_equal_keys_closed_form"]),
     "probe without 1/sqrt(d)": ("probe_scores", _probe_unscaled,
                                 ["test_probe_scores_match_sdpa_with_identity_values"]),
+    "probe heads grouped modulo": (
+        "probe_scores", _source_with(_ORIG_PROBE, "        g = h // G", "        g = h % Hkv"),
+        ["test_probe_scores_match_sdpa_with_identity_values"]),
+    "probe mask applied after the softmax": (
+        "probe_scores", _probe_mask_after_softmax,
+        ["test_probe_scores_match_sdpa_with_identity_values",
+         "test_probe_scores_invariants_and_equal_keys_closed_form"]),
     "ltp squared norm": ("ltp_scores", _ltp_squared,
                          ["test_ltp_identity_proxy_is_leading_norm", "test_ltp_matches_torch_on_exact_intermediates"]),
     "top-m one short": ("ltp_topm_scores", _topm_one_short, ["test_ltp_topm_brute_force_and_limits"]),
