@@ -274,6 +274,17 @@ MUTANTS = {
     "stage prune keeps the lowest scores": ("stage_prune", _stage_prune_lowest,
                                             ["test_stage_prune_worked_example",
                                              "test_msdp_prunes_by_the_last_layers_fused_score"]),
+    "active-row keys at the candidates' positions": (
+        "layer_forward",
+        _layer_with("reduced_attention(q_sel, pos[idx_a], kk[idx_a], vv[idx_a], pos[idx_a])",
+                    "reduced_attention(q_sel, pos[idx_a], kk[idx_a], vv[idx_a], pos[:len(idx_a)])"),
+        ["test_layer_kv_active_attention_is_dense_attention_of_the_active_rows",
+         "test_layer_kv_active_keep_all_equals_dense_layer"]),
+    "active-row flag ignored": (
+        "layer_forward",
+        _layer_with("    if cfg.kv_active:", "    if False:"),
+        ["test_layer_kv_active_attention_is_dense_attention_of_the_active_rows",
+         "test_layer_kv_active_keep_all_equals_dense_layer"]),
     "MSDP prunes by the stage's first layer": (
         "msdp_forward",
         _source_with(OS.msdp_forward, "            h, f = layer_forward(h, pos, layers[li], cfg, tr)",
