@@ -28,6 +28,12 @@ def _rmsnorm_wrong_axis(x, w=None, eps=1e-5):
     return y if w is None else y * np.asarray(w, dtype=np.float64)
 
 
+def _rmsnorm_eps_outside_root(x, w=None, eps=1e-5):
+    x = np.asarray(x, dtype=np.float64)
+    y = x / (np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) + eps)
+    return y if w is None else y * np.asarray(w, dtype=np.float64)
+
+
 def _rmsnorm_drops_weight(x, w=None, eps=1e-5):
     return _ORIG["rmsnorm"](x, None, eps)
 
@@ -215,10 +221,22 @@ _LAYER_PINS = ["test_layer_keep_all_equals_dense_layer", "test_layer_skipped_row
 
 
 _ORIG_PROBE = OS.probe_scores
+_ORIG_BF16 = OS.bf16_round
 
 # name -> (oracle function, mutant, pins that cover it)
 MUTANTS = {
     "rmsnorm over the wrong axis": ("rmsnorm", _rmsnorm_wrong_axis, ["test_rmsnorm_matches_torch"]),
+    "bf16 ties rounded away from zero": (
+        "bf16_round",
+        _source_with(_ORIG_BF16, "np.rint(np.ldexp(xf, -q))", "np.trunc(np.ldexp(xf, -q) + np.copysign(0.5, xf))"),
+        ["test_bf16_round_matches_torch_on_fp32_values"]),
+    "bf16 truncates": (
+        "bf16_round", _source_with(_ORIG_BF16, "np.rint(np.ldexp(xf, -q))", "np.trunc(np.ldexp(xf, -q))"),
+        ["test_bf16_round_matches_torch_on_fp32_values"]),
+    "bf16 keeps one bit too few": (
+        "bf16_round", _source_with(_ORIG_BF16, "q = np.maximum(e - 8, -133)", "q = np.maximum(e - 7, -133)"),
+        ["test_bf16_round_matches_torch_on_fp32_values"]),
+    "rmsnorm eps outside the root": ("rmsnorm", _rmsnorm_eps_outside_root, ["test_rmsnorm_matches_torch"]),
     "rmsnorm drops its weight": ("rmsnorm", _rmsnorm_drops_weight, ["test_rmsnorm_matches_torch"]),
     "rope turns backwards": ("rope", _rope_backwards,
                              ["test_rope_rotate_half_closed_form", "test_rope_matches_complex_rotation_and_is_relative"]),
