@@ -66,3 +66,22 @@ def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch)
     assert bench.captured_traffic("layer_32k") is None
     (src_dir / "attn.cu").write_text(text)
     assert bench.captured_traffic("layer_32k") == got
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` (the oracle on the host cores) prints one
+    JSON line with the contract's keys, on a small workload."""
+    import json
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "layer_small", "--steps", "1", "--warmup", "0"],
+                         capture_output=True, text=True, timeout=300, check=True).stdout
+    lines = [ln for ln in out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"]
+    assert d["metric"] == bench.METRIC and d["config"]["workload"] == "layer_small"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
