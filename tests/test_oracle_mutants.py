@@ -222,6 +222,8 @@ _LAYER_PINS = ["test_layer_keep_all_equals_dense_layer", "test_layer_skipped_row
 
 _ORIG_PROBE = OS.probe_scores
 _ORIG_BF16 = OS.bf16_round
+_ORIG_TOPM = OS.ltp_topm_scores
+_ORIG_FFN = OS.reduced_ffn
 
 # name -> (oracle function, mutant, pins that cover it)
 MUTANTS = {
@@ -260,6 +262,18 @@ MUTANTS = {
          "test_probe_scores_invariants_and_equal_keys_closed_form"]),
     "ltp squared norm": ("ltp_scores", _ltp_squared,
                          ["test_ltp_identity_proxy_is_leading_norm", "test_ltp_matches_torch_on_exact_intermediates"]),
+    "top-m sums the smallest": (
+        "ltp_topm_scores",
+        _source_with(_ORIG_TOPM, "np.sort(y, axis=1)[:, y.shape[1] - m:]", "np.sort(y, axis=1)[:, :m]"),
+        ["test_ltp_topm_brute_force_and_limits"]),
+    "top-m of signed values": (
+        "ltp_topm_scores",
+        _source_with(_ORIG_TOPM, "y = np.abs(t @ np.asarray(B, dtype=np.float64).T)",
+                     "y = t @ np.asarray(B, dtype=np.float64).T"),
+        ["test_ltp_topm_brute_force_and_limits"]),
+    "FFN gate and up swapped": (
+        "reduced_ffn", _source_with(_ORIG_FFN, "act = bf16_round(_silu(g) * u)", "act = bf16_round(_silu(u) * g)"),
+        ["test_reduced_ffn_rows_match_torch_swiglu"]),
     "top-m one short": ("ltp_topm_scores", _topm_one_short, ["test_ltp_topm_brute_force_and_limits"]),
     "fusion weights swapped": ("fuse_scores", _fuse_weights_swapped,
                                ["test_fuse_modes_exact_values", "test_fuse_std_add_is_weighted_zscores"]),

@@ -416,6 +416,8 @@ def test_layer_selection_wiring(w_a, w_b):
     assert np.array_equal(tr["idx_attn"], want_a)
     assert np.array_equal(np.nonzero(np.any(tr["h_attn"] != h, axis=1))[0], want_a)
     c = O.ltp_scores(O.bf16_round(O.rmsnorm(tr["h_attn"], W.norm_ffn, cfg.eps)), W.ltp_a, W.ltp_b)
+    # the LTP score itself, not only its ranking, is that of RMSNorm(h')
+    np.testing.assert_allclose(tr["c"], c, rtol=1e-12, atol=0)
     want_f = _top_k_rows(c.astype(np.float32), 12, 3) if w_a == 0 else want_a
     assert np.array_equal(tr["idx_ffn"], want_f)
     assert np.array_equal(np.nonzero(np.any(out != tr["h_attn"], axis=1))[0], want_f)
