@@ -224,6 +224,8 @@ _ORIG_PROBE = OS.probe_scores
 _ORIG_BF16 = OS.bf16_round
 _ORIG_TOPM = OS.ltp_topm_scores
 _ORIG_FFN = OS.reduced_ffn
+_ORIG_RESIDUAL = OS.attention_residual
+_ORIG_SALIENCE = OS.inject_salience
 
 # name -> (oracle function, mutant, pins that cover it)
 MUTANTS = {
@@ -291,6 +293,15 @@ MUTANTS = {
     "attention heads grouped modulo": ("reduced_attention", _attention_heads_modulo,
                                        ["test_reduced_attention_matches_sdpa_rows"]),
     "O projection untransposed": ("attention_residual", _residual_untransposed, ["test_attention_residual_rows"]),
+    "O projection without the bf16 operand": (
+        "attention_residual",
+        _source_with(_ORIG_RESIDUAL, "o = bf16_round(np.asarray(o_sel, dtype=np.float64).reshape(len(idx), -1))",
+                     "o = np.asarray(o_sel, dtype=np.float64).reshape(len(idx), -1) * (1 + 2.0 ** -9)"),
+        ["test_attention_residual_rows"]),
+    "salience grouped by the wrong heads": (
+        "inject_salience",
+        _source_with(_ORIG_SALIENCE, "mean = q_probe[:, g * G:(g + 1) * G, :]", "mean = q_probe[:, g::Hkv, :]"),
+        ["test_inject_salience_closed_form"]),
     "FFN with relu": ("reduced_ffn", _ffn_relu, ["test_reduced_ffn_rows_match_torch_swiglu"]),
     "FFN without its norm": ("reduced_ffn", _ffn_unnormalised, ["test_reduced_ffn_rows_match_torch_swiglu"]),
     "LTP scores the rows before attention": (

@@ -521,6 +521,17 @@ def test_inject_salience_closed_form():
     want[[1, 3], 0, 0] = torch.tensor(add, dtype=torch.float32).to(torch.bfloat16).item()
     want[[1, 3], 0, 1] = want[1, 0, 0]
     np.testing.assert_array_equal(out, want)
+    # two KV groups of two heads each (heads 0-1 read group 0, heads 2-3
+    # group 1): each group's keys move along its own heads' mean direction
+    q = np.zeros((1, 4, 4))
+    q[0, 0:2, 0] = 1.0
+    q[0, 2:4, 1] = 1.0
+    k = np.zeros((3, 2, 4))
+    out = O.inject_salience(k, q, np.array([2]), 2.0, 2)
+    want = np.zeros_like(k)
+    want[2, 0, 0] = 2.0
+    want[2, 1, 1] = 2.0
+    np.testing.assert_array_equal(out, want)
 
 
 # ---------------------------------------------------------------- accounting
