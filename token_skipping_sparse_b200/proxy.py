@@ -29,7 +29,7 @@ from __future__ import annotations
 
 import torch
 
-__all__ = ["ffn_outputs", "reduced_rank_fit", "derive_ltp_proxy"]
+__all__ = ["ffn_outputs", "reduced_rank_fit", "calibration_inputs", "derive_ltp_proxy"]
 
 
 def ffn_outputs(x, w_gate, w_up, w_down):
@@ -56,25 +56,35 @@ def reduced_rank_fit(X, Y, r, ridge=1e-4):
     return A, B, explained
 
 
+def calibration_inputs(D, n_samples=8192, seed=0, offset=1.0, device="cpu"):
+    """Synthetic FFN inputs [n_samples, D]: a fixed random offset direction
+    (scaled by ``offset``) plus N(0, 1) noise, each row scaled to unit RMS."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    mean = torch.randn(1, D, generator=g, device=device, dtype=torch.float32) * offset
+    X = mean + torch.randn(n_samples, D, generator=g, device=device, dtype=torch.float32)
+    return X / X.pow(2).mean(dim=1, keepdim=True).sqrt()      # unit RMS rows, as after RMSNorm
+
+
 def derive_ltp_proxy(w_gate, w_up, w_down, r, d_low=None, n_samples=8192, seed=0, ridge=1e-4, offset=1.0,
-                     chunk=2048):
+                     chunk=2048, X=None, exact=False):
     """Fit the LTP proxy of one FFN.
 
     Returns (A [r, D] bf16, B [d_low, r] bf16, channels [d_low] int64,
     explained) where ``explained`` is the share of the selected channels'
-    output energy that the rank-r proxy reproduces on the samples.
+    output energy that the rank-r proxy reproduces on the samples.  ``X``
+    replaces the drawn calibration inputs; ``exact`` returns A and B in fp64.
     """
     dev = w_gate.device
-    D = w_gate.shape[1]
-    g = torch.Generator(device=dev)
-    g.manual_seed(int(seed))
-    mean = torch.randn(1, D, generator=g, device=dev, dtype=torch.float32) * offset
-    X = mean + torch.randn(n_samples, D, generator=g, device=dev, dtype=torch.float32)
-    X = X / X.pow(2).mean(dim=1, keepdim=True).sqrt()      # unit RMS rows, as after RMSNorm
-    Y = torch.cat([ffn_outputs(X[i:i + chunk], w_gate, w_up, w_down) for i in range(0, n_samples, chunk)])
+    if X is None:
+        X = calibration_inputs(w_gate.shape[1], n_samples, seed, offset, dev)
+    n = X.shape[0]
+    Y = torch.cat([ffn_outputs(X[i:i + chunk], w_gate, w_up, w_down) for i in range(0, n, chunk)])
     if d_low is None or d_low >= Y.shape[1]:
         channels = torch.arange(Y.shape[1], device=dev)
-    else:
-        channels = torch.topk(Y.pow(2).sum(dim=0), d_low).indices.sort().values
+    else:  # the d_low channels of largest output energy, equal energies to the lower channel
+        channels = torch.argsort(-Y.double().pow(2).sum(dim=0), stable=True)[:d_low].sort().values
     A, B, explained = reduced_rank_fit(X, Y[:, channels], r, ridge)
+    if exact:
+        return A, B, channels, explained
     return A.to(torch.bfloat16), B.to(torch.bfloat16), channels, explained
