@@ -232,6 +232,13 @@ SPTS_API size_t spts_stage_prune_workspace(int64_t Nc);
  *    on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.
+ *  - CUDA loads device code lazily (the default module loading mode): the
+ *    first call on a device loads the code that holds the array and the
+ *    kernels it launches, which does take device memory.  A call with
+ *    Nc == 0 (every pointer may be NULL) is the set-up form: it only does
+ *    that per-device work on the current device and returns SPTS_OK.  A
+ *    caller that reserves the GPU's memory makes it once per device first;
+ *    after it, calls take no device memory at all.
  *  - Every call shares the one array, which keeps the last call's contents:
  *    calls that may overlap on the GPU (different streams, or different host
  *    threads on one device) race on it and must be serialised by the caller.

@@ -52,9 +52,9 @@ def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch)
     summary = os.path.join(root, "profiles", "attention_bf16_layer_32k.md")
     if not os.path.exists(summary):
         return
-    got = bench.captured_traffic("layer_32k")
+    got = bench.captured_traffic("layer_32k", "reduced_attention")
     assert got is not None and got > 0
-    assert bench.captured_traffic("no_such_workload") is None
+    assert bench.captured_traffic("no_such_workload", "reduced_attention") is None
     # a copy of the tree whose kernel source differs by one byte: no figure
     (tmp_path / "profiles").mkdir()
     shutil.copy(summary, tmp_path / "profiles" / "attention_bf16_layer_32k.md")
@@ -63,9 +63,9 @@ def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch)
     text = open(os.path.join(root, "token_skipping_sparse_b200", "csrc", "attn.cu")).read()
     (src_dir / "attn.cu").write_text(text + "\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.captured_traffic("layer_32k") is None
+    assert bench.captured_traffic("layer_32k", "reduced_attention") is None
     (src_dir / "attn.cu").write_text(text)
-    assert bench.captured_traffic("layer_32k") == got
+    assert bench.captured_traffic("layer_32k", "reduced_attention") == got
 
 
 def test_reference_arm_prints_one_contract_line():
@@ -85,3 +85,17 @@ def test_reference_arm_prints_one_contract_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    # the GPU arm's config object, key for key
+    from synthetic import WORKLOADS
+    wl = WORKLOADS["layer_small"]
+    assert d["config"] == bench.layer_config(wl, wl.k, 1)
+    assert "scaled" in cb["sample"] and "not scaled" in cb["sample"]
+
+
+def test_cpu_baseline_times_one_whole_layer():
+    from synthetic import WORKLOADS
+    wl = WORKLOADS["layer_small"]
+    cb = bench.cpu_baseline(wl)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
+    assert abs(cb["value"] * cb["seconds"] - wl.N) <= 0.05 * wl.N   # seconds is rounded to 1 ms
+    assert "unavailable" in bench.cpu_baseline(WORKLOADS["layer_small_kv"])

@@ -6,7 +6,8 @@ import pytest
 import torch
 
 import oracle as O
-from tests.gpu_util import assert_bf16_close, assert_close, band_check, np64
+from tests.gpu_util import assert_close, np64
+from tests.layer_check import check_layer_step, f64w, gpu_layer_step
 
 pytestmark = pytest.mark.gpu
 
@@ -107,53 +108,20 @@ def test_layer_norm_weights(shared):
 
 
 def _check_layer(wl, h, W, sal, pos, Wd):
-    desc = S.layer_desc(wl.D, wl.Hq, wl.Hkv, wl.d, wl.F, wl.r, wl.P, wl.k, fuse=wl.fuse,
-                        salient_rows=sal.cuda(), salient_shift=wl.salient_shift, ltp_dout=wl.ltp_dout, ltp_top_m=wl.ltp_top_m, seq_pool=0,
-                        kv_active_only=wl.kv_active)
+    """Every step of the layer on its own inputs (tests/layer_check.py), all
+    rows; then the oracle's uninterrupted chain, reported as drift."""
     hd = h.cuda()
-    out = S.spts_layer_forward(hd, pos.cuda(), desc, Wd, outputs=True)
-    S.check_device_status()
-    ow = O.LayerWeights(**{n: np64(t) for n, t in W.items()})
+    g, _ = gpu_layer_step(S, wl, hd, pos.cuda(), Wd, wl.k, sal.cuda() if len(sal) else None)
+    drift = {}
+    Wn = f64w(W)
+    ties = check_layer_step(wl, g, Wn, wl.k, sal=sal.numpy(), n_rows=None, drift=drift, label=wl.name)
+    ow = O.LayerWeights(**Wn)
     cfg = O.LayerConfig(Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, P=wl.P, k=wl.k, fuse=wl.fuse,
                         salient_rows=sal.numpy(), salient_shift=wl.salient_shift, kv_active=wl.kv_active,
                         ltp_top_m=wl.ltp_top_m)
     tr = {}
     O.layer_forward(np64(h), pos.numpy(), ow, cfg, tr)
-    s = out["s"].cpu().numpy()
-    assert_close(s, tr["s"], 1e-3 * tr["s"].max(), "probe scores")
-    ia = out["idx_attn"].cpu().numpy()
-    band_check(ia, tr["idx_attn"], tr["s"], tr["tau_attn"])
-    # reduced attention rows: oracle computes every row, compare at the GPU's picks
-    pn = pos.numpy()
-    q_all = O.bf16_round(O.rope((tr["xn"] @ ow.w_q.T).reshape(wl.N, wl.Hq, wl.d), pn))
-    if wl.kv_active:  # the keys are the GPU's active rows
-        o_sel = O.bf16_round(O.reduced_attention(q_all[ia], pn[ia], tr["k"][ia], tr["v"][ia], pn[ia]))
-    else:
-        o_sel = O.bf16_round(O.reduced_attention(q_all, pn, tr["k"], tr["v"], pn))[ia]
-    assert_bf16_close(np64(out["o_sel"]), o_sel, 2e-2, "o_sel")
-    ha = np64(out["h_attn"])
-    same = np.array_equal(ia, tr["idx_attn"])
-    if same:
-        assert_close(ha, tr["h_attn"], 2e-2, "h after attention")
-    # a8-a10 from the GPU's own h' (each step checked on the same input): LTP
-    # within the per-call bound, then the fused score and the FFN set exactly
-    # (the same fp32 operations on the same scores), then the reduced FFN
-    x2 = O.bf16_round(O.rmsnorm(ha, ow.norm_ffn, cfg.eps))
-    c_want = (O.ltp_topm_scores(x2, ow.ltp_a, ow.ltp_b, wl.ltp_top_m) if wl.ltp_top_m
-              else O.ltp_scores(x2, ow.ltp_a, ow.ltp_b))
-    c = out["c"].cpu().numpy()
-    assert_close(c, c_want, 1e-3 * c_want.max(), "ltp scores")
-    idf = out["idx_ffn"].cpu().numpy()
-    if wl.fuse == O.FUSE_SEQUENTIAL:  # the pool by s, then the k by c; f is c
-        assert np.array_equal(out["f"].cpu().numpy(), c)
-        want_f = O.select_sequential(s.astype(np.float32), c.astype(np.float32), min(wl.N, 2 * wl.k), wl.k, wl.P)[0]
-        assert np.array_equal(idf, want_f), "FFN selection"
-    else:
-        f_want = O.fuse_scores(s.astype(np.float32), c.astype(np.float32), wl.fuse, 0.5, 0.5)
-        assert np.array_equal(out["f"].cpu().numpy().view(np.uint32), f_want.view(np.uint32)), "fused score"
-        assert np.array_equal(idf, O.select_topk(f_want, wl.k, wl.P)[0]), "FFN selection"
-    h_want = O.reduced_ffn(ha, idf, ow.norm_ffn, cfg.eps, ow.w_gate, ow.w_up, ow.w_down)
-    assert_close(np64(hd), h_want, 2e-2, "h out (reduced FFN on the GPU's h')")
-    # the composed layer against the oracle's own chain: two bf16-stored stages
-    if same and np.array_equal(idf, tr["idx_ffn"]):
-        assert_close(np64(hd), tr["h_out"], 4e-2, "h out (composed)")
+    same = (np.array_equal(g["idx_attn"].numpy(), tr["idx_attn"])
+            and np.array_equal(g["idx_ffn"].numpy(), tr["idx_ffn"]))
+    chain = float(np.abs(g["h_out"].numpy() - tr["h_out"]).max()) if same else None
+    print(f"{wl.name}: {ties} near-tie differences; drift {drift}; whole-layer drift {chain}")

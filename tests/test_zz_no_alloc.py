@@ -5,14 +5,20 @@ plugin inside a host framework that reserved all GPU memory up front, or a
 latency-critical loop that cannot take cudaMalloc's implicit
 synchronisation.  For them spts_stage_prune_noalloc keeps its index scratch
 in a fixed device array inside the library.  These tests call it through the
-C ABI twice in a row and compare each result with the workspace-based
-spts_stage_prune on the same inputs; the results are integer indices and
-copied rows, so they must match exactly.  This file is named to run last.
+C ABI and compare it with the workspace-based spts_stage_prune on the same
+inputs, and with the oracle's stage prune; the results are integer indices
+and copied rows, so they must match exactly.  The calls come in pairs on one
+device -- the larger first, so the smaller one meets stale indices past its
+k_keep in the shared array -- with and without caller-supplied kept indices.
+After the set-up call (Nc == 0), repeated calls must leave the device's free
+memory unchanged.  This file is named to run last.
 """
 
 import numpy as np
 import pytest
 import torch
+
+import oracle as O
 
 pytestmark = pytest.mark.gpu
 
@@ -29,15 +35,53 @@ def _case(Nc, D, seed):
     return scores.cuda(), h.cuda(), pos.cuda()
 
 
-def test_noalloc_prune_matches_workspace_prune_on_two_calls():
-    for Nc, D, keep, tail, seed in [(100000, 64, 30000, 64, 1), (5000, 256, 1234, 16, 2)]:
-        scores, h, pos = _case(Nc, D, seed)
-        want_h, want_pos, want_kept = S.spts_stage_prune(scores, keep, tail, h, pos)
-        got_h, got_pos = S.spts_stage_prune_noalloc(scores, keep, tail, h, pos)
-        torch.cuda.synchronize()
-        assert torch.equal(got_pos, want_pos)
-        assert torch.equal(got_h, want_h)
-        assert torch.equal(pos[want_kept.long()], got_pos)
+def _setup():
+    S.check(S.lib.spts_stage_prune_noalloc(None, 0, 0, 0, None, None, 0, None, None, None, S.stream_ptr()))
+
+
+def _raw_call(scores, keep, tail, h, pos, h_out, pos_out, kept=None):
+    """The C entry point with caller-owned outputs (nothing allocated here)."""
+    return S.lib.spts_stage_prune_noalloc(S.ptr(scores), scores.shape[0], keep, tail, S.ptr(h), S.ptr(pos),
+                                          h.shape[1], S.ptr(h_out), S.ptr(pos_out), S.ptr(kept), S.stream_ptr())
+
+
+CASES = [(100000, 64, 30000, 64, 1), (5000, 256, 1234, 16, 2)]   # the larger call first
+
+
+def test_noalloc_prune_matches_workspace_prune_and_oracle_on_two_calls():
+    _setup()
+    for use_kept in (False, True):
+        for Nc, D, keep, tail, seed in CASES:
+            scores, h, pos = _case(Nc, D, seed)
+            want_h, want_pos, want_kept = S.spts_stage_prune(scores, keep, tail, h, pos)
+            kept = torch.full((keep,), -1, dtype=torch.int32, device="cuda") if use_kept else None
+            got_h, got_pos = S.spts_stage_prune_noalloc(scores, keep, tail, h, pos, kept=kept)
+            torch.cuda.synchronize()
+            assert torch.equal(got_pos, want_pos)
+            assert torch.equal(got_h, want_h)
+            if use_kept:
+                assert torch.equal(kept, want_kept)
+            # the oracle's prune: top-k_keep by score, tail forced, ties to the lower index
+            o_h, o_pos, o_kept = O.stage_prune(scores.cpu().numpy(), keep, tail, h.cpu().numpy(), pos.cpu().numpy())
+            assert np.array_equal(got_pos.cpu().numpy(), o_pos)
+            assert np.array_equal(got_h.cpu().numpy(), o_h)
+
+
+def test_noalloc_prune_takes_no_device_memory_after_setup():
+    Nc, D, keep, tail, seed = CASES[0]
+    scores, h, pos = _case(Nc, D, seed)
+    h_out = torch.empty(keep, D, device="cuda")
+    pos_out = torch.empty(keep, dtype=torch.int32, device="cuda")
+    _setup()
+    S.check(_raw_call(scores, keep, tail, h, pos, h_out, pos_out))
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(5):
+        S.check(_raw_call(scores, keep, tail, h, pos, h_out, pos_out))
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    want_h, want_pos, _ = S.spts_stage_prune(scores, keep, tail, h, pos)
+    assert torch.equal(h_out, want_h) and torch.equal(pos_out, want_pos)
 
 
 def test_noalloc_prune_rejects_oversize_and_leaves_context_usable():

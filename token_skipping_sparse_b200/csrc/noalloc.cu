@@ -14,6 +14,13 @@
 // `g_prune_scratch` is only a host-side stand-in, not a device address, so
 // the device address is looked up once per device with cudaGetSymbolAddress
 // (with that device current) and cached.
+//
+// CUDA loads device code lazily by default: the module holding the array is
+// loaded on that first address lookup, and each kernel on its first launch
+// or attribute query, and both take device memory.  A call with Nc == 0 is
+// the set-up form: it does the lookup and loads the two kernels the prune
+// launches, then returns, so a caller that reserves the GPU's memory makes it
+// once per device before the reservation.
 #include <mutex>
 
 #include "host.hpp"
@@ -52,6 +59,12 @@ extern "C" spts_status spts_stage_prune_noalloc(const float *scores, int64_t Nc,
                                                 const float *h_in, const int32_t *pos_in, int D, float *h_out,
                                                 int32_t *pos_out, int32_t *kept_idx, spts_stream stream) {
   const char *who = "spts_stage_prune_noalloc";
+  if (Nc == 0) {  // set-up only: resolve the array on this device, load the kernels
+    int32_t *p = nullptr;
+    SPTS_TRY(scratch_address(&p));
+    SPTS_TRY(preload_select_topk());
+    return preload_gather_rows();
+  }
   SPTS_REQUIRE(scores && h_in && pos_in && h_out && pos_out, SPTS_ERR_INVALID, "%s: NULL argument", who);
   SPTS_REQUIRE(Nc <= SPTS_NOALLOC_MAX_NC, SPTS_ERR_SHAPE,
                "%s: Nc = %lld exceeds the fixed scratch of %d candidates; use spts_stage_prune with a workspace",

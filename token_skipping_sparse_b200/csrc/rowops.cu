@@ -195,6 +195,12 @@ spts_status launch_gather_rows(const void *src, int64_t n_src, const int32_t *ro
   return SPTS_OK;
 }
 
+spts_status preload_gather_rows() {
+  cudaFuncAttributes a;
+  SPTS_CUDA_TRY(cudaFuncGetAttributes(&a, gather_rows_kernel));
+  return SPTS_OK;
+}
+
 // ---------------------------------------------------------------- salience
 // Synthetic-workload step (not SPTS): K[rows[t], g] += shift * unit(mean of
 // the group's probe queries).  Blocks (KV head, chunk of SAL_ROWS rows) of

@@ -51,6 +51,11 @@ spts_status launch_inject_salience(void *k, int64_t Nc, const void *q_probe, int
                                    const int32_t *rows, int64_t n_rows, float shift, uint32_t *status,
                                    cudaStream_t s);
 spts_status launch_gather_i32(const int32_t *src, const int32_t *idx, int64_t m, int32_t *dst, cudaStream_t s);
+// Load the kernels of the row gather / the top-k selection on the current
+// device now (CUDA loads a kernel's code lazily, at its first launch or
+// attribute query), so that a later launch takes no device memory for code.
+spts_status preload_gather_rows();
+spts_status preload_select_topk();
 spts_status launch_iota_i32(int32_t *dst, int64_t n, cudaStream_t s);
 spts_status launch_sum_groups(const float *group, int G, int64_t n, float *s, cudaStream_t st);
 

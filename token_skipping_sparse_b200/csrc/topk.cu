@@ -643,12 +643,9 @@ spts_status launch_select_topk(const float *s_a, const float *s_b, int mode, flo
   }
   if (n_free <= TK_SMEM_KEYS) {
     const size_t smem = static_cast<size_t>(n_free > 0 ? n_free : 1) * sizeof(uint32_t);
-    static bool attr = false;
-    if (!attr) {
-      SPTS_CUDA_TRY(cudaFuncSetAttribute(select_topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         TK_SMEM_KEYS * sizeof(uint32_t)));
-      attr = true;
-    }
+    // the attribute is per device: set it on every call (a few microseconds of host time)
+    SPTS_CUDA_TRY(cudaFuncSetAttribute(select_topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       TK_SMEM_KEYS * sizeof(uint32_t)));
     select_topk_kernel<true><<<1, TK_THREADS, smem, s>>>(fa, Nc, k, force_tail, idx_out, fused_out, kth_out,
                                                          status);
     note_launch();
@@ -658,6 +655,13 @@ spts_status launch_select_topk(const float *s_a, const float *s_b, int mode, flo
     note_launch();
   }
   SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+spts_status preload_select_topk() {
+  cudaFuncAttributes a;
+  SPTS_CUDA_TRY(cudaFuncGetAttributes(&a, select_topk_kernel<true>));
+  SPTS_CUDA_TRY(cudaFuncGetAttributes(&a, select_topk_kernel<false>));
   return SPTS_OK;
 }
 
