@@ -28,8 +28,10 @@
 //               packed fp32x2 FFMA before exp2, row sums in packed fp32x2
 //               adds, bf16 P back to TMEM; at the end O / l -> bf16.
 // Tile A holds the earlier tokens, so its key range is a prefix of B's: the
-// MMA and the softmax of A stop at A's own last visible key.  Pairs are
-// launched latest-first so the long ones start early.
+// MMA and the softmax of A stop at A's own last visible key.  CTAs run in
+// groups of HEAD_GROUP KV heads (the K/V they walk then fits in L2); inside a
+// group pairs are launched latest-first so the long ones start early.  Part
+// of each softmax row's exp2 runs on the FMA pipe (exp2_poly2).
 // All barrier waits are bounded (see sm100.cuh).
 #include <climits>
 
@@ -55,12 +57,23 @@ constexpr int OFF_BAR = OFF_V + KV_STAGES * TILE_BYTES;
 constexpr size_t SMEM_BYTES = OFF_BAR + 256;
 constexpr uint32_t TMEM_COLS = 512;  // S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+// One column pair in POLY_EVERY takes its exp2 from the polynomial on the
+// FMA pipe (exp2_poly2), the others from the MUFU pipe, which alone would
+// need as many cycles per key tile as the tile's two MMAs.
+#ifndef SPTS_ATTN_POLY_EVERY
+#define SPTS_ATTN_POLY_EVERY 3
+#endif
+constexpr int POLY_EVERY = SPTS_ATTN_POLY_EVERY;
+// KV heads per scheduling group: CTAs run group by group (pairs latest-first
+// inside a group), so the K/V that resident CTAs walk is the group's alone
+// and stays in L2 instead of being fetched from HBM several times.
+constexpr int HEAD_GROUP = 2;
 
 struct Params {
   const int32_t *qpos;
   const int32_t *kpos;
   __nv_bfloat16 *o;
-  int m, Nc, Hq, Hkv, G, tq, n_pairs;
+  int m, Nc, Hq, Hkv, G, tq, n_pairs, hgroup;
   float scale_log2;
   uint32_t *status;
   uint64_t wait_ns;
@@ -72,26 +85,8 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Packed fp32 pairs (sm_100a f32x2 arithmetic) and a three-input max: they
-// halve the instruction count of the softmax's per-element work.
-__device__ __forceinline__ uint64_t f2pack(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void f2unpack(uint64_t v, float &a, float &b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
+// A three-input max: with the packed f32x2 arithmetic of sm100.cuh it
+// halves the instruction count of the softmax's per-element work.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -113,8 +108,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   int *s_range = reinterpret_cast<int *>(tmem_holder + 2);  // per tile X: kv_end[X], mask_from[X]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / p.Hkv;
-  const int g = static_cast<int>(blockIdx.x) % p.Hkv;
+  const int per_group = p.n_pairs * p.hgroup;
+  const int rem = static_cast<int>(blockIdx.x) % per_group;
+  const int pair = p.n_pairs - 1 - rem / p.hgroup;
+  const int g = static_cast<int>(blockIdx.x) / per_group * p.hgroup + rem % p.hgroup;
   const int t0 = pair * 2 * p.tq;  // first token of tile A; tile B starts at t0 + tq
 
   if (smem_u32(smem) & 1023u) {
@@ -352,11 +349,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          float a0, a1;
-          f2unpack(f2fma(f2pack(__uint_as_float(xr[h * 64 + 2 * t]), __uint_as_float(xr[h * 64 + 2 * t + 1])), cc,
-                         mm),
-                   a0, a1);
-          const float e0 = ex2(a0), e1 = ex2(a1);
+          const uint64_t a2 =
+              f2fma(f2pack(__uint_as_float(xr[h * 64 + 2 * t]), __uint_as_float(xr[h * 64 + 2 * t + 1])), cc, mm);
+          float e0, e1;
+          if (t % POLY_EVERY == POLY_EVERY - 1) {  // this pair on the FMA pipe
+            exp2_poly2(a2, e0, e1);
+          } else {
+            float a0, a1;
+            f2unpack(a2, a0, a1);
+            e0 = ex2(a0);
+            e1 = ex2(a1);
+          }
           s4[t & 3] = f2add(s4[t & 3], f2pack(e0, e1));
           pk[t] = pack_bf16x2(e0, e1);
         }
@@ -451,6 +454,7 @@ spts_status launch_attention_bf16(const void *q, const int32_t *qpos, int64_t m,
   p.G = G;
   p.tq = tq;
   p.n_pairs = static_cast<int>((m + 2 * tq - 1) / (2 * tq));
+  p.hgroup = Hkv % HEAD_GROUP == 0 ? HEAD_GROUP : 1;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = status;
   p.wait_ns = wait_limit_ns();

@@ -410,6 +410,56 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Packed fp32 pairs (sm_100a f32x2 arithmetic): one instruction for two
+// values on the FMA pipe.
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x for a pair of x <= 0 on the FMA and integer pipes, leaving the MUFU
+// (exp2) pipe to the other elements of a softmax row.  Range reduction:
+// x = j + f with j = round(x) (adding 1.5 * 2^23 leaves round(x) in the low
+// mantissa bits) and f in [-1/2, 1/2]; 2^f by the degree-3 polynomial of
+// smallest maximum relative error on that interval (7.5e-5; coefficients
+// derived by exp2_poly_fit.py beside this package); j goes into the exponent
+// field by an integer add.  x is clamped at -125 so the exponent stays
+// normal: a masked (-inf) element gives 2^-125 instead of 0, which no bf16
+// probability or fp32 row sum can tell from zero next to the row's maximum
+// (which contributes 1).
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float &e0, float &e1) {
+  float a, b;
+  f2unpack(x2, a, b);
+  const uint64_t x = f2pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t shifter = f2pack(12582912.f, 12582912.f);  // 1.5 * 2^23
+  const uint64_t y = f2add(x, shifter);
+  const uint64_t j = f2add(y, f2pack(-12582912.f, -12582912.f));
+  const uint64_t f = f2fma(j, f2pack(-1.f, -1.f), x);
+  uint64_t p = f2fma(f2pack(0.0551716685295105f, 0.0551716685295105f), f,
+                     f2pack(0.2426111251115799f, 0.2426111251115799f));
+  p = f2fma(p, f, f2pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2fma(p, f, f2pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, y0, y1;
+  f2unpack(p, p0, p1);
+  f2unpack(y, y0, y1);
+  e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(y0) << 23));
+  e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23));
+}
+
 // Byte offset of 16-byte unit `u` (0..7) of row `r` inside a 128-byte-swizzled
 // tile whose rows are 128 bytes (the layout TMA SWIZZLE_128B writes and UMMA
 // SW128 reads; the tile base must be 1024-byte aligned).
