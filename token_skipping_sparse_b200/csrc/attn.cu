@@ -102,7 +102,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t *sV = smem + OFF_V;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = k_full + KV_STAGES, *kv_empty = v_full + KV_STAGES,
-           *s_full = kv_empty + KV_STAGES, *p_ready = s_full + 2, *o_done = p_ready + 2, *drain = o_done + 2;
+           *s_full = kv_empty + KV_STAGES, *p_ready = s_full + 2, *o_done = p_ready + 4, *drain = o_done + 2;
+  // p_ready[2 X + h]: P of tile X for keys [64 h, 64 h + 64) is in TMEM
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
   int *s_range = reinterpret_cast<int *>(tmem_holder + 2);  // per tile X: kv_end[X], mask_from[X]
@@ -127,7 +128,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
-      mbar_init(&p_ready[x], 128);
+      mbar_init(&p_ready[2 * x], 128);
+      mbar_init(&p_ready[2 * x + 1], 128);
       mbar_init(&o_done[x], 1);
     }
     mbar_init(drain, 1);
@@ -227,16 +229,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_commit_w(&s_full[x]);
         return true;
       };
+      // PV in two halves of 64 keys, each issued as soon as the softmax has
+      // stored that half of P: the first half runs while the softmax is
+      // still on the second.
       auto issue_pv = [&](int x, int j) -> bool {
         const int st = j % KV_STAGES;
-        if (!wait_all(&p_ready[x], j & 1, 0x24u)) return false;
         if (!wait_all(&v_full[st], (j / KV_STAGES) & 1, 0x25u)) return false;
-        tc_fence_after();
         const uint32_t v_addr = smem_u32(sV + st * TILE_BYTES);
+        for (int half = 0; half < 2; ++half) {
+          if (!wait_all(&p_ready[2 * x + half], j & 1, 0x24u)) return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t v = sdesc_mn_sw128(v_addr + kk * 16 * 128, CHUNK_BYTES);
-          mma_bf16_ts_w(tmem + 256 + x * 128, tmem + x * BKV + kk * 8, v, idesc_pv, (j | kk) != 0);
+          for (int kq = 0; kq < 4; ++kq) {
+            const int kk = 4 * half + kq;
+            const uint64_t v = sdesc_mn_sw128(v_addr + kk * 16 * 128, CHUNK_BYTES);
+            mma_bf16_ts_w(tmem + 256 + x * 128, tmem + x * BKV + kk * 8, v, idesc_pv, (j | kk) != 0);
+          }
         }
         tc_commit_w(&o_done[x]);
         return true;
@@ -365,6 +373,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         // P over this tile's S values: columns [32h, 32h+32) hold keys [64h, 64h+64)
         tmem_st32(lane_base + s_col + h * 32, pk);
+        if (h == 0) {  // the first half of P is in place: its PV can start
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&p_ready[2 * x]);
+        }
       }
       {
         float q0, q1, q2, q3, q4, q5, q6, q7;
@@ -375,7 +388,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_ready[x]);
+      mbar_arrive(&p_ready[2 * x + 1]);
     }
     // final normalisation once the last PV of this tile has landed
     if (ok && n_tiles > 0) {
