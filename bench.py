@@ -17,7 +17,8 @@ region is bracketed by barriers and the time is the max over ranks.
 
 The default line (``--workload layer_32k``) also carries the metric's second
 configuration, the 128K layer, as its ``layer_128k`` object (``--no-128k``
-leaves it out).  Roofline fractions divide by the burst bf16 peak of
+leaves it out), and a few 32K prefills of the 32-layer Table B schedule with
+their TTFT ratio against keep 1.0 as ``llama32_32k`` (``--no-schedule``).  Roofline fractions divide by the burst bf16 peak of
 MEASURED_PEAKS.json (the timed regions are short and run at full clock); the
 sustained fraction is reported beside it.
 
@@ -365,57 +366,63 @@ def measure_layer(S, wl, args, rank, world, dev, peaks, e2e=True):
         del hd
 
     # ---------------- end to end through the C ABI with host buffers
-    e2e_res = None
+    e2e_res = e2e_f32 = None
     if not msdp and e2e:
-        hh = torch.empty_like(lcase.h0, device="cpu").pin_memory()
-        hh.copy_(lcase.h0.cpu())
-        ho = torch.empty_like(hh).pin_memory()
-        # Consecutive steps are pipelined the way a caller streaming sequences
-        # would run them: NBUF device buffers, the H2D copy, the layer call and
-        # the D2H copy on three streams, so step i's copies overlap the
-        # neighbouring steps' compute (PCIe runs both directions at once).
-        # A buffer cycles through H2D, compute and D2H, so with three of them
-        # the copy engines, not the buffer count, bound the rate.
-        # Every step still moves its own input in and its result out.
-        NBUF = 3
-        ne = min(steps, 10)
-        dbuf = [torch.empty_like(lcase.h0) for _ in range(NBUF)]
-        s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-        ev_in = [torch.cuda.Event() for _ in range(NBUF)]
-        ev_done = [torch.cuda.Event() for _ in range(NBUF)]
-        ev_free = [torch.cuda.Event() for _ in range(NBUF)]
+        def run_e2e(io_bf16):
+            # Consecutive steps are pipelined the way a caller streaming
+            # sequences would run them: NBUF device buffers, the H2D copy, the
+            # layer call and the D2H copy on three streams, so step i's copies
+            # overlap the neighbouring steps' compute (PCIe runs both
+            # directions at once).  Every step moves its own input in and its
+            # result out.  io_bf16: the residual crosses the boundary in bf16
+            # (spts_layer_forward_bf16io), else in fp32 (spts_layer_forward).
+            dt = torch.bfloat16 if io_bf16 else torch.float32
+            hh = lcase.h0.to(dt).cpu().pin_memory()
+            ho = torch.empty_like(hh).pin_memory()
+            NBUF = 3
+            ne = min(steps, 10)
+            dbuf = [torch.empty_like(lcase.h0, dtype=dt) for _ in range(NBUF)]
+            s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+            ev_in = [torch.cuda.Event() for _ in range(NBUF)]
+            ev_done = [torch.cuda.Event() for _ in range(NBUF)]
+            ev_free = [torch.cuda.Event() for _ in range(NBUF)]
+            call = S.spts_layer_forward_bf16io if io_bf16 else S.spts_layer_forward
 
-        def pipelined(n):
-            for i in range(n):
-                b = i % NBUF
-                if i >= NBUF:
-                    s_in.wait_event(ev_free[b])        # the buffer's previous result is out
-                with torch.cuda.stream(s_in):
-                    dbuf[b].copy_(hh, non_blocking=True)
-                    ev_in[b].record(s_in)
-                s_cmp.wait_event(ev_in[b])
-                with torch.cuda.stream(s_cmp):
-                    S.spts_layer_forward(dbuf[b], lcase.pos, desc, lcase.weights)
-                    ev_done[b].record(s_cmp)
-                s_out.wait_event(ev_done[b])
-                with torch.cuda.stream(s_out):
-                    ho.copy_(dbuf[b], non_blocking=True)
-                    ev_free[b].record(s_out)
+            def pipelined(n):
+                for i in range(n):
+                    b = i % NBUF
+                    if i >= NBUF:
+                        s_in.wait_event(ev_free[b])        # the buffer's previous result is out
+                    with torch.cuda.stream(s_in):
+                        dbuf[b].copy_(hh, non_blocking=True)
+                        ev_in[b].record(s_in)
+                    s_cmp.wait_event(ev_in[b])
+                    with torch.cuda.stream(s_cmp):
+                        call(dbuf[b], lcase.pos, desc, lcase.weights)
+                        ev_done[b].record(s_cmp)
+                    s_out.wait_event(ev_done[b])
+                    with torch.cuda.stream(s_out):
+                        ho.copy_(dbuf[b], non_blocking=True)
+                        ev_free[b].record(s_out)
 
-        pipelined(NBUF)
-        torch.cuda.synchronize()
-        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        x0.record(s_in)
-        pipelined(ne)
-        x1.record(s_out)                              # after the last step's D2H
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(x0.elapsed_time(x1) / ne, dev)
-        nbh = hh.numel() * hh.element_size()
-        e2e_res = {"value": round(wl.N * world / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": nbh,
-                   "d2h_bytes_per_step": nbh, "ms_per_step": round(e2e_ms, 4),
-                   "pipeline": f"{NBUF} device buffers; H2D, layer call and D2H on separate streams, overlapping "
-                               "across consecutive steps"}
-        del dbuf, hh, ho
+            pipelined(NBUF)
+            torch.cuda.synchronize()
+            x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            x0.record(s_in)
+            pipelined(ne)
+            x1.record(s_out)                              # after the last step's D2H
+            torch.cuda.synchronize()
+            e_ms = max_over_ranks(x0.elapsed_time(x1) / ne, dev)
+            nbh = hh.numel() * hh.element_size()
+            return {"value": round(wl.N * world / (e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": nbh,
+                    "d2h_bytes_per_step": nbh, "ms_per_step": round(e_ms, 4),
+                    "boundary": ("bf16 residual (spts_layer_forward_bf16io: fp32 inside, changed rows rounded "
+                                 "back to bf16)") if io_bf16 else "fp32 residual (spts_layer_forward)",
+                    "pipeline": f"{NBUF} device buffers; H2D, layer call and D2H on separate streams, overlapping "
+                                "across consecutive steps"}
+
+        e2e_res = run_e2e(True)
+        e2e_f32 = run_e2e(False)
 
     traffic = captured_traffic(wl.name, dom)
     out = {
@@ -438,6 +445,7 @@ def measure_layer(S, wl, args, rank, world, dev, peaks, e2e=True):
         "gpu_launches": int(launches),
         "clocks": clocks,
         "e2e": e2e_res,
+        "e2e_fp32_boundary": e2e_f32,
         "dense_keep1": dense,
     }
     del keep_alive
@@ -461,6 +469,21 @@ def gpu_arm(args, rank, world, dev):
     if args.workload == "layer_32k" and not args.no_128k:
         sub = measure_layer(S, WORKLOADS["layer_128k"], args, rank, world, dev, peaks, e2e=not args.no_e2e)
         result["layer_128k"] = sub
+    # the 32-layer Table B schedule at 32K (a few prefills): TTFT against keep 1.0
+    if args.workload == "layer_32k" and not args.no_schedule:
+        sargs = argparse.Namespace(**{**vars(args), "workload": "llama32_32k", "steps": 3, "warmup": 1})
+        sch = schedule_arm(sargs, rank, world, dev)
+        jac = [j["jaccard"] for j in sch["jaccard_consecutive"]]
+        result["llama32_32k"] = {
+            "what": "32 LLaMA-shaped layers under the Table B schedule, one step = one 32K prefill",
+            "steps": sch["steps"], "warmup": sch["warmup"], "ttft_ms": sch["ttft_ms"],
+            "ttft_ratio_vs_keep1": sch["ttft_ratio_vs_keep1"], "value": sch["value"], "unit": sch["unit"],
+            "roofline_frac": sch["roofline"]["frac"], "layer_roofline_frac": sch["layer_roofline"]["frac"],
+            "jaccard_consecutive_mean": round(float(np.mean(jac)), 4) if jac else None,
+            "jaccard_consecutive_min": round(float(np.min(jac)), 4) if jac else None,
+            "rows_after_prefill": sch["rows_after_prefill"], "gpu_launches": sch["gpu_launches"],
+            "clocks": sch["clocks"]}
+        torch.cuda.empty_cache()
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl)
     return result
@@ -640,6 +663,47 @@ def schedule_arm(args, rank, world, dev):
     }
 
 
+def attention_arm(args, rank, world, dev):
+    """spts_reduced_attention alone on a workload's shapes: seeded bf16
+    N(0,1) Q/K/V, positions 0..N-1, the selected rows a seeded random subset
+    with the last P kept.  For profiling one kernel at a size that holds about
+    a gigabyte on the device (the whole 128K layer holds several)."""
+    import token_skipping_sparse_b200 as S
+    wl = WORKLOADS[args.workload]
+    peaks = measured_peaks()
+    g = torch.Generator().manual_seed(wl.seed + 11)
+    k = wl.k
+    sel = torch.cat([torch.sort(torch.randperm(wl.N - wl.P, generator=g)[:k - wl.P]).values,
+                     torch.arange(wl.N - wl.P, wl.N)]).to(torch.int32)
+    q = torch.randn(k, wl.Hq, wl.d, generator=g).to(torch.bfloat16).to(dev)
+    kk = torch.randn(wl.N, wl.Hkv, wl.d, generator=g).to(torch.bfloat16).to(dev)
+    vv = torch.randn(wl.N, wl.Hkv, wl.d, generator=g).to(torch.bfloat16).to(dev)
+    pos = torch.arange(wl.N, dtype=torch.int32, device=dev)
+    qpos = sel.to(dev)
+    o = torch.empty_like(q)
+    for _ in range(args.warmup):
+        S.spts_reduced_attention(q, qpos, kk, vv, pos, out=o)
+    torch.cuda.synchronize()
+    S.check_device_status()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        S.spts_reduced_attention(q, qpos, kk, vv, pos, out=o)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    flops = 4.0 * wl.Hq * wl.d * float((sel.to(torch.float64) + 1.0).sum())
+    ach = flops / (ms / 1e3) / 1e12
+    return {"metric": "reduced attention TFLOP/s (kernel alone)", "value": round(ach, 1), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) Q/K/V, random selection)",
+            "config": {"workload": wl.name, "kernel": "reduced_attention", "N": wl.N, "k": k, "Hq": wl.Hq,
+                       "Hkv": wl.Hkv, "d_head": wl.d},
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                         "frac": round(ach / peaks["bf16"], 4), "traffic": None}}
+
+
 def reference_arm(args):
     """The oracle (fp32 timed mode) on the host cores: one whole layer per
     step, on the GPU arm's workload, config, metric and unit."""
@@ -681,6 +745,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-128k", action="store_true", help="time only the 32K layer in the default line")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) measurement")
+    ap.add_argument("--no-schedule", action="store_true", help="leave the 32-layer schedule out of the default line")
+    ap.add_argument("--kernel", default=None, choices=["attention"],
+                    help="time one kernel alone on the workload's shapes (for profiling)")
     args = ap.parse_args()
     if args.steps is None:
         base = args.workload.rsplit("_", 1)[0]  # a variant takes its base workload's count
@@ -701,7 +768,12 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                              device_id=dev)
     try:
-        res = schedule_arm(args, rank, world, dev) if WORKLOADS[args.workload].schedule else gpu_arm(args, rank, world, dev)
+        if args.kernel == "attention":
+            res = attention_arm(args, rank, world, dev)
+        elif WORKLOADS[args.workload].schedule:
+            res = schedule_arm(args, rank, world, dev)
+        else:
+            res = gpu_arm(args, rank, world, dev)
     finally:
         if world > 1:
             torch.distributed.barrier()

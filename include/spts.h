@@ -121,6 +121,13 @@ SPTS_API uint64_t spts_debug_get_wait_limit_ns(void);
  * devices, all threads); a measurement aid. */
 SPTS_API uint64_t spts_launch_count(void);
 
+/* Testing hook: y[i] = the exp2 that the reduced-attention softmax kernel
+ * evaluates on the FMA pipe for part of each row (range reduction to
+ * 2^round(x) * 2^f, a degree-3 polynomial in f with p(0) = 1, relative error
+ * <= 1.02e-4 for -126 <= x <= 0; exactly 0 for x <= -127 and -inf), on
+ * device arrays x, y [n] fp32. */
+SPTS_API spts_status spts_debug_exp2_poly(const float *x, int64_t n, float *y, spts_stream stream);
+
 /* ---------------------------------------------------------------------- */
 /* The six calls of the hot path                                          */
 /* ---------------------------------------------------------------------- */
@@ -145,6 +152,9 @@ SPTS_API size_t spts_probe_scores_workspace(const spts_attn_desc *a, int P, int6
  * scores[i] = || (x_i A^T) B^T ||_2 with the rank-r intermediate kept in bf16.
  *   x [Nc, D] bf16 (the FFN input, i.e. already normalized), A [r, D] bf16,
  *   B [Dout, r] bf16, scores [Nc] fp32 out.
+ * Evaluated as sqrt(t G t^T), t = bf16(x_i A^T), with the Gram matrix
+ * G = B^T B built on each call in the workspace (2 * r^2 bf16 + 8 * r^2 fp32):
+ * the same value up to rounding, at r x r instead of r x Dout per row.
  * Limits: dt = SPTS_BF16; D % 64 == 0; r % 64 == 0, 64 <= r <= 256;
  * Dout % 256 == 0. */
 SPTS_API spts_status spts_ltp_scores(spts_dtype dt, const void *x, int64_t Nc, int D, const void *A, int r,
@@ -352,6 +362,8 @@ typedef struct {
   int32_t *idx_ffn;    /* [k] rows that ran the reduced FFN      */
   void *o_sel;         /* [k, Hq, d] bf16 reduced-attention out  */
   float *h_attn;       /* [Nc, D] residual after attention       */
+  void *k;             /* [Nc, Hkv, d] bf16 keys after RoPE (and the synthetic salience): the probe's keys */
+  void *q_probe;       /* [P, Hq, d] bf16 probe queries after RoPE */
   /* NULL, or an array of SPTS_LAYER_STAGE_EVENTS cudaEvent_t handles
    * created by the caller, any of which may be NULL (not recorded); event i
    * is recorded on the stream after stage i (see below), event 0 before the
@@ -379,6 +391,20 @@ SPTS_API spts_status spts_layer_forward(const spts_layer_desc *L, const spts_lay
                                const int32_t *pos, int64_t Nc, const spts_layer_outputs *out, void *ws,
                                size_t ws_bytes, spts_stream stream);
 SPTS_API size_t spts_layer_forward_workspace(const spts_layer_desc *L, int64_t Nc);
+
+/* spts_layer_forward on a residual stream held in bf16 at the boundary:
+ * h [Nc, D] bf16, in place.  The layer runs on an fp32 copy of h in the
+ * workspace (the same kernels and results as spts_layer_forward on
+ * float(h)); then the rows it changed -- its attention rows and FFN rows,
+ * every row when L->k == Nc -- are rounded to bf16 (nearest even) back into
+ * h, and the rows it skipped keep their input bits.  This halves what a
+ * caller moves across PCIe when h lives in host memory.  `out` as for
+ * spts_layer_forward (h_attn, when given, is the fp32 residual after
+ * attention).  Limits: those of spts_layer_forward; D % 8 == 0. */
+SPTS_API spts_status spts_layer_forward_bf16io(const spts_layer_desc *L, const spts_layer_weights *W, void *h,
+                                               const int32_t *pos, int64_t Nc, const spts_layer_outputs *out,
+                                               void *ws, size_t ws_bytes, spts_stream stream);
+SPTS_API size_t spts_layer_forward_bf16io_workspace(const spts_layer_desc *L, int64_t Nc);
 
 /* Multi-Stage Delayed Pruning over a stack of layers (SPTS, Fig. 2(c),
  * Fig. A, Table B).  n_stages stages of layers_per_stage layers each

@@ -30,14 +30,15 @@ def assert_close(got, want, atol, what=""):
         f"{what}: max |err| {err.max():.3e} > {atol:.1e} at flat {i} (got {got.flat[i]!r}, want {want.flat[i]!r})"
 
 
-def assert_bf16_close(got, want, atol, what=""):
-    """bf16 outputs: within atol, or within one bf16 ulp of the oracle value
-    (a rounding flip between the fp32 kernel and the fp64 oracle)."""
+def assert_bf16_close(got, want, atol, what="", ulps=1):
+    """bf16 outputs: within atol, or within `ulps` bf16 ulps of the oracle
+    value (a rounding flip between the fp32 kernel and the fp64 oracle at
+    each of the `ulps` bf16 roundings the value went through)."""
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     ulp = np.where(want != 0, 2.0 ** (np.floor(np.log2(np.abs(want) + 1e-300)) - 7), 2.0 ** -133)
     err = np.abs(got - want)
-    bad = err > np.maximum(atol, ulp * 1.0001)
+    bad = err > np.maximum(atol, ulps * ulp * 1.0001)
     if bad.any():
         i = int(np.argmax(bad))
         raise AssertionError(f"{what}: {int(bad.sum())} elements off; first flat {i}: got {got.flat[i]!r} "

@@ -1,8 +1,9 @@
 """Teacher-forced parity of one SPTS layer (helper of the GPU tests; not collected).
 
 Every step of the layer is compared with the oracle on the inputs the GPU's
-step itself received: the probe scores and the attention rows from the
-layer's input h, the O projection from the GPU's own O_sel, the LTP score and
+step itself received: K and the probe queries from the layer's input h, the
+probe scores from the GPU's own K and probe queries, the attention rows from
+the layer's input h, the O projection from the GPU's own O_sel, the LTP score and
 the reduced FFN from the GPU's own h' (the output of the attention half), the
 fused score and both selections from the GPU's own scores.  So every gate is
 one call on the same inputs, at the per-call tolerance: 2e-2 max-abs for bf16
@@ -104,12 +105,29 @@ def check_layer_step(wl, g, Wn, k, sal=None, n_rows=None, seed=0, drift=None, la
     full = n_rows is None
     tag = f"{label}: " if label else ""
 
-    # a1-a4: norm, K/V, probe queries, probe scores, the MHA selection
+    # a1-a2: norm, K/V, probe queries.  K and the probe queries are bf16
+    # intermediates: within 2e-2 or one bf16 ulp of the oracle's (a rounding
+    # flip between the fp32 kernel and the fp64 oracle)
     xn, K, V = _norm_kv(wl, h, Wn, pos)
     qp = O.bf16_round(O.rope((xn[N - P:].astype(np.float64) @ Wn["w_q"].T).reshape(P, wl.Hq, wl.d), pos[N - P:]))
     if sal is not None and len(sal):
         K = O.inject_salience(K, qp, np.asarray(sal), wl.salient_shift, wl.Hkv)
-    s, _ = O.probe_scores(qp, pos[N - P:], K, pos)
+    gk = g["k"].float().numpy()
+    gqp = np64(g["q_probe"])
+    salient = np.zeros(N, bool)
+    if sal is not None and len(sal):
+        salient[np.asarray(sal)] = True
+    for a in range(0, N, 16384):
+        b = min(N, a + 16384)
+        plain = ~salient[a:b]
+        assert_bf16_close(gk[a:b][plain], K[a:b][plain], PER_CALL_TOL, tag + "K")
+        # salient keys are rounded to bf16 twice: after RoPE and after the shift
+        assert_bf16_close(gk[a:b][~plain], K[a:b][~plain], PER_CALL_TOL, tag + "K (salient rows)", ulps=2)
+    assert_bf16_close(gqp, qp, PER_CALL_TOL, tag + "probe queries")
+    # a3-a4: the probe scores on the GPU's own keys and probe queries (a
+    # one-ulp flip of one key element moves that key's weight in every probe
+    # row, so the oracle's own K would not be the same input), the MHA selection
+    s, _ = O.probe_scores(gqp, pos[N - P:], gk, pos)
     gs = g["s"].numpy()
     assert_close(gs, s, 1e-3 * s.max(), tag + "probe scores")
     assert abs(gs.astype(np.float64).sum() - P * wl.Hq) < 1e-3 * P * wl.Hq, tag + "probe score sum"

@@ -61,6 +61,8 @@ def _cases(S):
     bad_g = S.AttnDesc(S.BF16, 30, 8, 128, 0.0)      # Hq % Hkv != 0
     bad_d = S.AttnDesc(S.F32, 32, 8, 96, 0.0)        # head dim not 64 / 128
     g16 = S.AttnDesc(S.BF16, 32, 2, 128, 0.0)        # 16 query heads per KV head
+    ld = S.layer_desc(1024, 8, 2, 128, 1536, 64, 16, 300)
+    lw = S.LayerWeights(*([A16] * 9 + [None, None]))
     ref = ctypes.byref
     return [
         # probe scores: descriptor, P range, alignment
@@ -146,6 +148,13 @@ def _cases(S):
                                                     None), S.ERR_SHAPE, "N % 256"),
         ("salience geometry", lambda: lib.spts_inject_salience(A16, 10, B16, 4, 32, 8, 96, None, 0, 1.0, None),
          S.ERR_SHAPE, "geometry"),
+        # the layer on a bf16 residual: alignment of h, positions present
+        ("bf16io misaligned h", lambda: lib.spts_layer_forward_bf16io(ref(ld), ref(lw), M8, A16, 1000, None, None, 0,
+                                                                      None), S.ERR_INVALID, "bad h/pos"),
+        ("bf16io NULL pos", lambda: lib.spts_layer_forward_bf16io(ref(ld), ref(lw), A16, None, 1000, None, None, 0,
+                                                                  None), S.ERR_INVALID, "bad h/pos"),
+        ("bf16io k > Nc", lambda: lib.spts_layer_forward_bf16io(ref(ld), ref(lw), A16, B16, 200, None, None, 0,
+                                                                None), S.ERR_SHAPE, "P <= k <= Nc"),
     ]
 
 

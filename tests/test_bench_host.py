@@ -3,7 +3,6 @@ divides by (brute-force pair counts), and the ncu traffic figure it reports
 only while the captured kernel source is unchanged."""
 
 import os
-import shutil
 import types
 
 import numpy as np
@@ -48,24 +47,23 @@ def test_gemm_flops():
 
 
 def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch):
-    root = bench.ROOT
-    summary = os.path.join(root, "profiles", "attention_bf16_layer_32k.md")
-    if not os.path.exists(summary):
-        return
-    got = bench.captured_traffic("layer_32k", "reduced_attention")
-    assert got is not None and got > 0
-    assert bench.captured_traffic("no_such_workload", "reduced_attention") is None
-    # a copy of the tree whose kernel source differs by one byte: no figure
-    (tmp_path / "profiles").mkdir()
-    shutil.copy(summary, tmp_path / "profiles" / "attention_bf16_layer_32k.md")
+    """A tree whose kernel source matches the summary's recorded hash gets
+    the summary's DRAM figure; one byte of difference gives None."""
+    import hashlib
     src_dir = tmp_path / "token_skipping_sparse_b200" / "csrc"
     src_dir.mkdir(parents=True)
-    text = open(os.path.join(root, "token_skipping_sparse_b200", "csrc", "attn.cu")).read()
-    (src_dir / "attn.cu").write_text(text + "\n")
-    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.captured_traffic("layer_32k", "reduced_attention") is None
+    (tmp_path / "profiles").mkdir()
+    text = "// a kernel source\n"
     (src_dir / "attn.cu").write_text(text)
-    assert bench.captured_traffic("layer_32k", "reduced_attention") == got
+    sha = hashlib.sha256(text.encode()).hexdigest()[:16]
+    (tmp_path / "profiles" / "attention_bf16_layer_32k.md").write_text(
+        f"Source: attn.cu sha256 prefix `{sha}`.\n\n| DRAM read / write per launch | 215.8 MB / 59.9 MB |\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.captured_traffic("layer_32k", "reduced_attention") == round(275.7e6)
+    assert bench.captured_traffic("layer_128k", "reduced_attention") is None      # no capture
+    assert bench.captured_traffic("layer_32k", "gate_up_swiglu") is None          # no summary kind
+    (src_dir / "attn.cu").write_text(text + "\n")
+    assert bench.captured_traffic("layer_32k", "reduced_attention") is None
 
 
 def test_reference_arm_prints_one_contract_line():

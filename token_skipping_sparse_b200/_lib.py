@@ -34,6 +34,7 @@ EXPORTS = (
     "spts_stage_prune_workspace", "spts_stage_prune_noalloc", "spts_rmsnorm_rows", "spts_rope", "spts_gather_rows", "spts_linear",
     "spts_linear_workspace", "spts_inject_salience", "spts_layer_forward", "spts_layer_forward_workspace",
     "spts_msdp_forward", "spts_msdp_forward_workspace", "spts_schedule_forward", "spts_schedule_forward_workspace",
+    "spts_layer_forward_bf16io", "spts_layer_forward_bf16io_workspace", "spts_debug_exp2_poly",
 )
 
 
@@ -73,8 +74,8 @@ class LayerWeights(C.Structure):
 
 
 class LayerOutputs(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in ("s", "c", "f", "idx_attn", "idx_ffn", "o_sel", "h_attn",
-                                          "stage_events")]
+    _fields_ = [(n, C.c_void_p) for n in ("s", "c", "f", "idx_attn", "idx_ffn", "o_sel", "h_attn", "k",
+                                          "q_probe", "stage_events")]
 
 
 LAYER_STAGE_EVENTS = 16
@@ -97,6 +98,7 @@ _sig("spts_check_device_status", i32, [vp, vp])
 _sig("spts_debug_set_wait_limit_ns", None, [u64])
 _sig("spts_debug_get_wait_limit_ns", u64, [])
 _sig("spts_launch_count", u64, [])
+_sig("spts_debug_exp2_poly", i32, [vp, i64, vp, vp])
 _sig("spts_probe_scores", i32, [AD, vp, vp, i32, vp, vp, i64, vp, vp, vp, sz, vp])
 _sig("spts_probe_scores_workspace", sz, [AD, i32, i64])
 _sig("spts_ltp_scores", i32, [i32, vp, i64, i32, vp, i32, vp, i32, vp, vp, sz, vp])
@@ -128,6 +130,9 @@ if hasattr(lib, "spts_layer_forward"):
     _sig("spts_msdp_forward", i32, [C.POINTER(LayerDesc), C.POINTER(LayerWeights), i32, i32, C.POINTER(C.c_int64),
                                     i32, vp, vp, i64, vp, vp, sz, vp])
     _sig("spts_msdp_forward_workspace", sz, [C.POINTER(LayerDesc), i64])
+    _sig("spts_layer_forward_bf16io", i32, [C.POINTER(LayerDesc), C.POINTER(LayerWeights), vp, vp, i64,
+                                            C.POINTER(LayerOutputs), vp, sz, vp])
+    _sig("spts_layer_forward_bf16io_workspace", sz, [C.POINTER(LayerDesc), i64])
 _sig("spts_schedule_forward", i32, [C.POINTER(LayerDesc), C.POINTER(LayerWeights), i32, i32, C.POINTER(C.c_int),
                                     C.POINTER(C.c_int64), i32, i64, vp, vp, i64, C.POINTER(C.c_int64), vp, i64,
                                     C.POINTER(C.c_int64), vp, sz, vp])
@@ -180,6 +185,13 @@ def workspace(nbytes, device=None):
 
 def launch_count():
     return int(lib.spts_launch_count())
+
+
+def debug_exp2_poly(x):
+    """The reduced-attention softmax's FMA-pipe exp2 applied to a device fp32 tensor."""
+    y = torch.empty_like(x)
+    check(lib.spts_debug_exp2_poly(ptr(x), x.numel(), ptr(y), stream_ptr()))
+    return y
 
 
 def set_wait_limit_ns(ns):
@@ -410,7 +422,9 @@ def spts_layer_forward(h, pos, desc, weights, outputs=False, ws=None, events=Non
                    idx_attn=torch.empty(k, dtype=torch.int32, device=dv),
                    idx_ffn=torch.empty(k, dtype=torch.int32, device=dv),
                    o_sel=torch.empty(k, desc.Hq, desc.d, dtype=torch.bfloat16, device=dv),
-                   h_attn=torch.empty_like(h))
+                   h_attn=torch.empty_like(h),
+                   k=torch.empty(Nc, desc.Hkv, desc.d, dtype=torch.bfloat16, device=dv),
+                   q_probe=torch.empty(desc.P, desc.Hq, desc.d, dtype=torch.bfloat16, device=dv))
         for n, t in res.items():
             setattr(out, n, t.data_ptr())
     w = weights if isinstance(weights, LayerWeights) else layer_weights(weights)
@@ -419,6 +433,18 @@ def spts_layer_forward(h, pos, desc, weights, outputs=False, ws=None, events=Non
     check(lib.spts_layer_forward(C.byref(desc), C.byref(w), ptr(h), ptr(pos), Nc,
                                  None if out is None else C.byref(out), ptr(ws), ws.numel(), stream_ptr()))
     return res
+
+
+def spts_layer_forward_bf16io(h, pos, desc, weights, ws=None):
+    """One layer in place on a bf16 residual h [Nc, D]: computed in fp32 on
+    a workspace copy; the rows the layer changed are rounded back to bf16."""
+    Nc = h.shape[0]
+    w = weights if isinstance(weights, LayerWeights) else layer_weights(weights)
+    n = lib.spts_layer_forward_bf16io_workspace(C.byref(desc), Nc)
+    ws = workspace(n) if ws is None else ws
+    check(lib.spts_layer_forward_bf16io(C.byref(desc), C.byref(w), ptr(h), ptr(pos), Nc, None, ptr(ws), ws.numel(),
+                                        stream_ptr()))
+    return h
 
 
 def spts_msdp_forward(h, pos, desc, layer_weights_list, layers_per_stage, stage_k, stage_pos=False, ws=None):

@@ -75,7 +75,7 @@ spts_status spts_probe_scores(const spts_attn_desc *a, const void *q_probe, cons
 }
 
 // ------------------------------------------------------------------ LTP
-size_t spts_ltp_scores_workspace(int64_t, int, int, int) { return kStatusBytes; }
+size_t spts_ltp_scores_workspace(int64_t, int, int r, int) { return kStatusBytes + Carver::round(ltp_gram_bytes(r)); }
 
 spts_status spts_ltp_scores(spts_dtype dt, const void *x, int64_t Nc, int D, const void *A, int r, const void *B,
                             int Dout, float *scores, void *ws, size_t ws_bytes, spts_stream stream) {
@@ -91,7 +91,9 @@ spts_status spts_ltp_scores(spts_dtype dt, const void *x, int64_t Nc, int D, con
                "%s: misaligned pointer", who);
   SPTS_TRY(check_ws(ws, ws_bytes, spts_ltp_scores_workspace(Nc, D, r, Dout), who));
   if (Nc == 0) return SPTS_OK;
-  return launch_ltp_bf16(x, Nc, D, A, r, B, Dout, scores, static_cast<uint32_t *>(ws), cs(stream));
+  Carver cv(ws, ws_bytes);
+  void *gram = cv.take(ltp_gram_bytes(r));
+  return launch_ltp_bf16(x, Nc, D, A, r, B, Dout, scores, cv.status(), cs(stream), 0, gram);
 }
 
 size_t spts_ltp_topm_scores_workspace(int64_t, int, int, int) { return kStatusBytes; }
@@ -113,7 +115,7 @@ spts_status spts_ltp_topm_scores(spts_dtype dt, const void *x, int64_t Nc, int D
                "%s: misaligned pointer", who);
   SPTS_TRY(check_ws(ws, ws_bytes, spts_ltp_topm_scores_workspace(Nc, D, r, Dout), who));
   if (Nc == 0) return SPTS_OK;
-  return launch_ltp_bf16(x, Nc, D, A, r, B, Dout, scores, static_cast<uint32_t *>(ws), cs(stream), top_m);
+  return launch_ltp_bf16(x, Nc, D, A, r, B, Dout, scores, static_cast<uint32_t *>(ws), cs(stream), top_m, nullptr);
 }
 
 // ------------------------------------------------------------------ select
@@ -320,6 +322,14 @@ spts_status spts_inject_salience(void *k, int64_t Nc, const void *q_probe, int P
   SPTS_REQUIRE(Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && d > 0 && d <= 1024 && (d & (d - 1)) == 0 && P > 0,
                SPTS_ERR_SHAPE, "%s: bad geometry", who);
   return launch_inject_salience(k, Nc, q_probe, P, Hq, Hkv, d, rows, n_rows, shift, nullptr, cs(stream));
+}
+
+spts_status spts_debug_exp2_poly(const float *x, int64_t n, float *y, spts_stream stream) {
+  const char *who = "spts_debug_exp2_poly";
+  SPTS_REQUIRE(n >= 0, SPTS_ERR_SHAPE, "%s: n < 0", who);
+  SPTS_REQUIRE(n == 0 || (x && y), SPTS_ERR_INVALID, "%s: NULL argument", who);
+  SPTS_REQUIRE(aligned(x, 4) && aligned(y, 4), SPTS_ERR_INVALID, "%s: misaligned pointer", who);
+  return launch_exp2_poly(x, n, y, cs(stream));
 }
 
 }  // extern "C"

@@ -66,8 +66,13 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 constexpr int POLY_EVERY = SPTS_ATTN_POLY_EVERY;
 // KV heads per scheduling group: CTAs run group by group (pairs latest-first
 // inside a group), so the K/V that resident CTAs walk is the group's alone
-// and stays in L2 instead of being fetched from HBM several times.
+// and stays in L2 instead of being fetched from HBM several times.  Two
+// heads while their K/V (512 B per key and head) stays within ~48 MB, one
+// head beyond (a model of the dispatch with LRU over 64 KB K/V tiles and
+// ~60 MB of effective L2: 32K keys, two heads: 128 MB of K/V read, the
+// floor; 128K keys: 0.77 GB with one head against 1.5 GB with two).
 constexpr int HEAD_GROUP = 2;
+constexpr int64_t HEAD_GROUP_MAX_KEYS = 49152;
 
 struct Params {
   const int32_t *qpos;
@@ -467,7 +472,7 @@ spts_status launch_attention_bf16(const void *q, const int32_t *qpos, int64_t m,
   p.G = G;
   p.tq = tq;
   p.n_pairs = static_cast<int>((m + 2 * tq - 1) / (2 * tq));
-  p.hgroup = Hkv % HEAD_GROUP == 0 ? HEAD_GROUP : 1;
+  p.hgroup = (Hkv % HEAD_GROUP == 0 && Nc <= HEAD_GROUP_MAX_KEYS) ? HEAD_GROUP : 1;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = status;
   p.wait_ns = wait_limit_ns();

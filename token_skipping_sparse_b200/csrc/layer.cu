@@ -17,6 +17,7 @@ struct LayerBufs {
   int32_t *idx_a, *idx_f, *qpos;
   void *topk;  // scratch of the grid top-k
   void *ksel;  // K of the active rows (kv_active_only)
+  void *gram;  // the LTP proxy's Gram matrix (L2-norm score)
 };
 
 // Carves the workspace; with cv.base == nullptr it only measures.
@@ -41,6 +42,7 @@ void carve(Carver &cv, const spts_layer_desc *L, int64_t Nc, LayerBufs &b) {
   b.qpos = static_cast<int32_t *>(cv.take(k * 4));
   b.topk = cv.take(select_sequential_scratch_bytes(Nc));  // also covers the plain top-k
   b.ksel = cv.take(k * hk * 2);
+  b.gram = cv.take(L->F > 0 ? ltp_gram_bytes(L->r) : 1);
 }
 
 // A side stream and fork/join events per (host thread, device): the V and
@@ -172,7 +174,7 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   carve(cv, L, Nc, b);
   uint32_t *st = cv.status();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (L->k == Nc && !o.s && !o.c && !o.f && !o.idx_attn && !o.idx_ffn && L->n_salient == 0)
+  if (L->k == Nc && !o.s && !o.c && !o.f && !o.idx_attn && !o.idx_ffn && !o.k && !o.q_probe && L->n_salient == 0)
     return dense_layer(L, W, h, pos, Nc, o, b, st, s);
   const int D = L->D, P = L->P, hq = L->Hq * L->d, hk = L->Hkv * L->d;
   const int64_t k = L->k;
@@ -231,6 +233,9 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   if (L->n_salient > 0)
     SPTS_TRY(launch_inject_salience(b.kk, Nc, b.qprobe, P, L->Hq, L->Hkv, L->d, L->salient_rows, L->n_salient,
                                     L->salient_shift, st, s));
+  if (o.k) SPTS_CUDA_TRY(cudaMemcpyAsync(o.k, b.kk, static_cast<size_t>(Nc) * hk * 2, cudaMemcpyDeviceToDevice, s));
+  if (o.q_probe)
+    SPTS_CUDA_TRY(cudaMemcpyAsync(o.q_probe, b.qprobe, static_cast<size_t>(P) * hq * 2, cudaMemcpyDeviceToDevice, s));
   SPTS_TRY(mark(4));
 
   // a3-a4: probe scores, MHA selection
@@ -286,7 +291,7 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
     SPTS_TRY(launch_rmsnorm_rows(h, nullptr, Nc, D, W->norm_ffn, L->eps, b.xn, s));
   SPTS_TRY(mark(11));
   SPTS_TRY(launch_ltp_bf16(b.xn, Nc, D, W->ltp_a, L->r, W->ltp_b, L->ltp_dout > 0 ? L->ltp_dout : D, c, st, s,
-                           L->ltp_top_m));
+                           L->ltp_top_m, b.gram));
   SPTS_TRY(mark(12));
   if (L->fuse == SPTS_FUSE_SEQUENTIAL) {
     const int64_t pool = L->seq_pool > 0 ? L->seq_pool : std::min<int64_t>(Nc, 2 * k);
@@ -303,6 +308,52 @@ spts_status spts_layer_forward(const spts_layer_desc *L, const spts_layer_weight
   GemmArgs g2{b.act, k, L->F, W->w_down, nullptr, D, SPTS_EPI_SCATTER_ADD, h, idx_f, nullptr, 0.0, st};
   SPTS_TRY(launch_gemm(g2, s));
   return mark(15);
+}
+
+// ---------------------------------------------------------------- bf16 residual boundary
+// The layer on a bf16 residual stream at the boundary: h is converted to an
+// fp32 copy in the workspace, spts_layer_forward runs on the copy, and the
+// rows the layer changed (its attention rows and FFN rows; every row at
+// k == Nc) are rounded back to bf16 in place.  Rows it skipped are not
+// touched, so they keep their bf16 input exactly.
+size_t spts_layer_forward_bf16io_workspace(const spts_layer_desc *L, int64_t Nc) {
+  if (L == nullptr || Nc <= 0) return kStatusBytes;
+  return Carver::round(spts_layer_forward_workspace(L, Nc)) + Carver::round(static_cast<size_t>(Nc) * L->D * 4) +
+         2 * Carver::round(static_cast<size_t>(L->k > 0 ? L->k : 1) * 4);
+}
+
+spts_status spts_layer_forward_bf16io(const spts_layer_desc *L, const spts_layer_weights *W, void *h,
+                                      const int32_t *pos, int64_t Nc, const spts_layer_outputs *out, void *ws,
+                                      size_t ws_bytes, spts_stream stream) {
+  const char *who = "spts_layer_forward_bf16io";
+  SPTS_TRY(check_layer(L, W, Nc));
+  SPTS_REQUIRE(h && pos && aligned(h, 16) && aligned(pos, 4), SPTS_ERR_INVALID, "%s: bad h/pos", who);
+  SPTS_TRY(check_ws(ws, ws_bytes, spts_layer_forward_bf16io_workspace(L, Nc), who));
+  const size_t lw = Carver::round(spts_layer_forward_workspace(L, Nc));
+  char *extra = static_cast<char *>(ws) + lw;
+  float *hf = reinterpret_cast<float *>(extra);
+  extra += Carver::round(static_cast<size_t>(Nc) * L->D * 4);
+  int32_t *ia = reinterpret_cast<int32_t *>(extra);
+  int32_t *iff = reinterpret_cast<int32_t *>(extra + Carver::round(static_cast<size_t>(L->k > 0 ? L->k : 1) * 4));
+  uint32_t *st = static_cast<uint32_t *>(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  SPTS_TRY(launch_bf16_to_f32(h, Nc * L->D, hf, s));
+  spts_layer_outputs o;
+  if (out) o = *out;
+  else memset(&o, 0, sizeof(o));
+  const bool all_rows = L->k == Nc;  // keep 1.0: every row changes (and the dense path stays available)
+  if (!all_rows) {
+    if (!o.idx_attn) o.idx_attn = ia;
+    if (L->F > 0 && !o.idx_ffn) o.idx_ffn = iff;
+  }
+  SPTS_TRY(spts_layer_forward(L, W, hf, pos, Nc, &o, ws, lw, stream));
+  if (all_rows) {
+    SPTS_TRY(launch_iota_i32(ia, Nc, s));  // k == Nc: ia holds Nc entries
+    return launch_rows_f32_to_bf16(hf, ia, Nc, Nc, L->D, h, st, s);
+  }
+  SPTS_TRY(launch_rows_f32_to_bf16(hf, o.idx_attn, L->k, Nc, L->D, h, st, s));
+  if (L->F > 0) SPTS_TRY(launch_rows_f32_to_bf16(hf, o.idx_ffn, L->k, Nc, L->D, h, st, s));
+  return SPTS_OK;
 }
 
 // ---------------------------------------------------------------- MSDP

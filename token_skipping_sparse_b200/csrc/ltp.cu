@@ -6,17 +6,19 @@
 //   phase 1  T = X A^T   (M=128, N=r, K=D) accumulated in TMEM, then read
 //            back, rounded to bf16 and stored in shared memory in the UMMA
 //            K-major swizzled layout, where it becomes the A operand of
-//   phase 2  Y = T B^T   (M=128, N=256 per chunk, K=r), chunk by chunk over
-//            the Dout outputs into two ping-pong TMEM accumulators; the
-//            epilogue warps fold every chunk into a per-row sum of squares.
-// With top_m > 0 (D_low = Dout <= 512, both chunks resident in TMEM) the
+//   phase 2  for the L2 norm, U = T G with the Gram matrix G = B^T B (r x r,
+//            built per call, as two bf16 halves G_hi + G_lo): ||T B^T||^2 =
+//            rowsum(T * U), so phase 2 costs r x r instead of r x Dout per
+//            row (Dout = 4096, r = 256: 16x less); T stays in TMEM beside U.
+// With top_m > 0 (D_low = Dout <= 512) phase 2 is Y = T B^T (M=128, N=256 per
+// chunk, K=r), both chunks resident in TMEM, and the
 // score is instead the sum of the top_m largest |y| of the row (top-rho
 // channel saliency, Table E): each row's thread searches the float bits of
 // |y| from the top for a threshold with exactly top_m values at or above it
 // (counting passes over the row in TMEM, at most 31, usually about half),
 // then sums the values above it plus the ties at it that top_m needs.
-// Per row only 2*D bytes of X are read from HBM; A and B (2 x r x D bf16)
-// are shared by all CTAs through L2.  Waits are bounded.
+// Per row only 2*D bytes of X are read from HBM; A, B and G are shared by
+// all CTAs through L2.  Waits are bounded.
 #include "host.hpp"
 #include "rowops.cuh"
 #include "sm100.cuh"
@@ -35,7 +37,7 @@ constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 256;
 
 struct Params {
   int M, D, r, Dout;
-  int top_m;  // 0: L2 norm of y; > 0: sum of the top_m largest |y| (Dout <= 512)
+  int top_m;  // 0: L2 norm of y through the Gram form; > 0: sum of the top_m largest |y| (Dout <= 512)
   float *scores;
   uint32_t *status;
   uint64_t wait_ns;
@@ -43,7 +45,8 @@ struct Params {
 
 __global__ void __launch_bounds__(THREADS, 1)
     ltp_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
-               const __grid_constant__ CUtensorMap tmB, const __grid_constant__ Params p) {
+               const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmGhi,
+               const __grid_constant__ CUtensorMap tmGlo, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sT = smem + OFF_TS;
@@ -56,6 +59,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * 128;
   const int kb1 = p.D / 64, kb2 = p.r / 64, nch = p.Dout / 256;
+  const bool gram = p.top_m == 0;  // phase 2 against G_hi, then G_lo (r x r each)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -85,9 +89,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmX);
       tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmB);
+      if (gram) {
+        tma_prefetch_desc(&tmGhi);
+        tma_prefetch_desc(&tmGlo);
+      } else {
+        tma_prefetch_desc(&tmB);
+      }
       uint32_t issued = 0, par = 0;
-      const int total = kb1 + nch * kb2;
+      const int total = kb1 + (gram ? 2 * kb2 : nch * kb2);
       for (int i = 0; i < total; ++i) {
         const int st = i % STAGES;
         const uint32_t ph = (i / STAGES) & 1;
@@ -97,6 +106,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_arrive_expect_tx(&full[st], X_BYTES + p.r * 128);
           tma_load_2d(slot, &tmX, &full[st], i * 64, m0);
           tma_load_2d(slot + X_BYTES, &tmA, &full[st], i * 64, 0);
+        } else if (gram) {  // G_hi k-blocks, then G_lo k-blocks: r rows x 64 columns
+          const int j = i - kb1;
+          mbar_arrive_expect_tx(&full[st], p.r * 128);
+          tma_load_2d(slot, j < kb2 ? &tmGhi : &tmGlo, &full[st], (j % kb2) * 64, 0);
         } else {
           const int j = i - kb1;
           mbar_arrive_expect_tx(&full[st], 256 * 128);
@@ -134,7 +147,26 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ok) ok = mbar_wait(ts_ready, 0, abort_flag, p.status, p.wait_ns, 0x53u);
       tc_fence_after();
       const uint32_t t_addr = smem_u32(sT);
-      for (int nc = 0; ok && nc < nch; ++nc) {
+      if (gram && ok) {  // U = T G_hi^T + T G_lo^T into TMEM columns [256, 256 + r); T stays at [0, r)
+        const uint32_t idesc_g = idesc_bf16_f32(128, p.r, 0, 0);
+        for (int j = 0; ok && j < 2 * kb2; ++j, ++i) {
+          const int st = i % STAGES;
+          if (!mbar_wait(&full[st], (i / STAGES) & 1, abort_flag, p.status, p.wait_ns, 0x59u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int kb = j % kb2;
+          const uint32_t base = smem_u32(smem + st * SLOT);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tmem + 256, sdesc_k_sw128(t_addr + kb * CHUNK_BYTES) + 2 * kk, sdesc_k_sw128(base) + 2 * kk,
+                        idesc_g, (j | kk) != 0);
+          tc_commit(&empty[st]);
+        }
+        if (ok) tc_commit(&acc_full[0]);
+      }
+      for (int nc = 0; ok && !gram && nc < nch; ++nc) {
         const int acc = nc & 1;
         if (!mbar_wait(&acc_empty[acc], ((nc >> 1) & 1) ^ 1u, abort_flag, p.status, p.wait_ns, 0x54u)) break;
         tc_fence_after();
@@ -238,29 +270,24 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok && m0 + rr < p.M) p.scores[m0 + rr] = ss;
     }
-    for (int nc = 0; ok && p.top_m == 0 && nc < nch; ++nc) {
-      const int acc = nc & 1;
-      const bool okw = mbar_wait(&acc_full[acc], (nc >> 1) & 1, abort_flag, p.status, p.wait_ns, 0x57u);
-      if (!__all_sync(0xffffffffu, okw)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+    if (gram) {  // c^2 = sum_j bf16(T_j) U_j with U = bf16(T) G: T at [0, r), U at [256, 256 + r)
+      const bool okw = mbar_wait(&acc_full[0], 0, abort_flag, p.status, p.wait_ns, 0x5Au);
+      ok = ok && __all_sync(0xffffffffu, okw);
+      if (ok) {
+        tc_fence_after();
 #pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 32) {
-        uint32_t y[32];
-        tmem_ld32(lane_base + acc * 256 + c0, y);
-        tmem_ld_wait();
+        for (int c0 = 0; c0 < p.r; c0 += 32) {
+          uint32_t t[32], u[32];
+          tmem_ld32(lane_base + c0, t);
+          tmem_ld32(lane_base + 256 + c0, u);
+          tmem_ld_wait();
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const float v = __uint_as_float(y[t]);
-          ss = fmaf(v, v, ss);
+          for (int q = 0; q < 32; ++q)
+            ss = fmaf(__bfloat162float(__float2bfloat16_rn(__uint_as_float(t[q]))), __uint_as_float(u[q]), ss);
         }
+        if (m0 + rr < p.M) p.scores[m0 + rr] = sqrtf(fmaxf(ss, 0.f));
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[acc]);
     }
-    if (ok && p.top_m == 0 && m0 + rr < p.M) p.scores[m0 + rr] = sqrtf(ss);
   }
   __syncthreads();
   if (warp == 1) {
@@ -269,19 +296,132 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------- Gram form
+// For the L2-norm score ||t B^T||^2 = t (B^T B) t^T, so the second product
+// needs only the r x r Gram matrix G = B^T B instead of all Dout outputs.
+// G is built per call from B: fp32 partial sums of the upper-triangle 64 x 64
+// blocks over up to 32 slices of the Dout rows (products of two bf16 are
+// exact in fp32), then summed in a fixed slice order -- deterministic, and
+// symmetric by construction (the lower blocks are the upper ones mirrored)
+// -- and split into bf16 G_hi = bf16(G), G_lo = bf16(G - G_hi) for the
+// tensor core (G_hi + G_lo carries 16 significant bits).
+constexpr int GRAM_MAX_SPLITS = 32;
+constexpr int GRAM_ROWS = 32;  // B rows staged per step
+
+__host__ __device__ inline int gram_splits(int Dout) {  // slices of a multiple of GRAM_ROWS rows each
+  const int s = Dout / GRAM_ROWS;
+  return s < GRAM_MAX_SPLITS ? s : GRAM_MAX_SPLITS;
+}
+
+// Block (jb, kb), jb <= kb (G is symmetric), of 64 x 64 entries of G over the
+// rows of slice blockIdx.y; blockIdx.x enumerates the upper-triangle blocks.
+// 256 threads, 4 x 4 entries each; B rows staged in shared memory as fp32.
+__global__ void __launch_bounds__(256) gram_partial_kernel(const __nv_bfloat16 *__restrict__ B, int Dout, int r,
+                                                           int splits, float *__restrict__ part) {
+  __shared__ __align__(16) float sj[GRAM_ROWS][64];
+  __shared__ __align__(16) float sk[GRAM_ROWS][64];
+  const int nb = r / 64;
+  int jb = 0, t = blockIdx.x;
+  while (t >= nb - jb) {
+    t -= nb - jb;
+    ++jb;
+  }
+  const int kb = jb + t;
+  const int j0 = jb * 64, k0 = kb * 64;
+  const int rows = Dout / splits, o0 = blockIdx.y * rows;
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  const int lo = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;  // staging: row, first of 8 columns
+  float acc[4][4] = {};
+  for (int ob = 0; ob < rows; ob += GRAM_ROWS) {
+    const int64_t row = static_cast<int64_t>(o0 + ob + lo) * r;
+    const uint4 vj = *reinterpret_cast<const uint4 *>(B + row + j0 + lc);
+    const uint4 vk = *reinterpret_cast<const uint4 *>(B + row + k0 + lc);
+    const uint32_t wj[4] = {vj.x, vj.y, vj.z, vj.w}, wk[4] = {vk.x, vk.y, vk.z, vk.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // bf16 -> fp32 is a 16-bit shift
+      sj[lo][lc + 2 * q] = __uint_as_float(wj[q] << 16);
+      sj[lo][lc + 2 * q + 1] = __uint_as_float(wj[q] & 0xFFFF0000u);
+      sk[lo][lc + 2 * q] = __uint_as_float(wk[q] << 16);
+      sk[lo][lc + 2 * q + 1] = __uint_as_float(wk[q] & 0xFFFF0000u);
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int o = 0; o < GRAM_ROWS; ++o) {
+      const float4 a4 = *reinterpret_cast<const float4 *>(&sj[o][ty * 4]);
+      const float4 b4 = *reinterpret_cast<const float4 *>(&sk[o][tx * 4]);
+      const float a[4] = {a4.x, a4.y, a4.z, a4.w}, b[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[q][w] = fmaf(a[q], b[w], acc[q][w]);
+    }
+    __syncthreads();
+  }
+  float *dst = part + static_cast<int64_t>(blockIdx.y) * r * r;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<float4 *>(dst + (j0 + ty * 4 + q) * r + k0 + tx * 4) =
+        make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
+}
+
+// G[j][k] = sum of the slices in order (entries below the diagonal blocks
+// read their mirror), then G_hi = bf16(G), G_lo = bf16(G - G_hi).
+__global__ void gram_finish_kernel(const float *__restrict__ part, int r, int splits, __nv_bfloat16 *__restrict__ g_hi,
+                                   __nv_bfloat16 *__restrict__ g_lo) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= r * r) return;
+  int j = i / r, k = i % r;
+  if (j / 64 > k / 64) {
+    const int t = j;
+    j = k;
+    k = t;
+  }
+  float g = 0.f;
+  for (int s = 0; s < splits; ++s) g += part[static_cast<int64_t>(s) * r * r + j * r + k];
+  const __nv_bfloat16 hi = __float2bfloat16_rn(g);
+  g_hi[i] = hi;
+  g_lo[i] = __float2bfloat16_rn(g - __bfloat162float(hi));
+}
+
 }  // namespace
 
+size_t ltp_gram_bytes(int r) {
+  const size_t rr = static_cast<size_t>(r > 0 ? r : 1) * (r > 0 ? r : 1);
+  auto up = [](size_t n) { return (n + 255) / 256 * 256; };
+  return 2 * up(rr * 2) + up(static_cast<size_t>(GRAM_MAX_SPLITS) * rr * 4);
+}
+
 spts_status launch_ltp_bf16(const void *x, int64_t Nc, int D, const void *A, int r, const void *B, int Dout,
-                            float *scores, uint32_t *status, cudaStream_t s, int top_m) {
+                            float *scores, uint32_t *status, cudaStream_t s, int top_m, void *gram_ws) {
   if (Nc == 0) return SPTS_OK;
-  CUtensorMap tx, ta, tb;
+  CUtensorMap tx, ta, tb, tghi, tglo;
   SPTS_TRY(tmap_bf16_2d(&tx, x, static_cast<uint64_t>(Nc), D, D, 128));
   SPTS_TRY(tmap_bf16_2d(&ta, A, r, D, D, static_cast<uint32_t>(r)));
   SPTS_TRY(tmap_bf16_2d(&tb, B, Dout, r, r, 256));
+  if (top_m == 0) {  // the Gram form: G = B^T B, then its bf16 halves
+    SPTS_REQUIRE(gram_ws != nullptr, SPTS_ERR_WORKSPACE, "ltp: no scratch for the Gram matrix");
+    const size_t rr = static_cast<size_t>(r) * r;
+    auto up = [](size_t n) { return (n + 255) / 256 * 256; };
+    uint8_t *w = static_cast<uint8_t *>(gram_ws);
+    __nv_bfloat16 *g_hi = reinterpret_cast<__nv_bfloat16 *>(w);
+    __nv_bfloat16 *g_lo = reinterpret_cast<__nv_bfloat16 *>(w + up(rr * 2));
+    float *part = reinterpret_cast<float *>(w + 2 * up(rr * 2));
+    const int nb = r / 64, splits = gram_splits(Dout);
+    gram_partial_kernel<<<dim3(nb * (nb + 1) / 2, splits), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(B), Dout,
+                                                                        r, splits, part);
+    note_launch();
+    gram_finish_kernel<<<static_cast<unsigned>((rr + 255) / 256), 256, 0, s>>>(part, r, splits, g_hi, g_lo);
+    note_launch();
+    SPTS_TRY(tmap_bf16_2d(&tghi, g_hi, r, r, r, static_cast<uint32_t>(r)));
+    SPTS_TRY(tmap_bf16_2d(&tglo, g_lo, r, r, r, static_cast<uint32_t>(r)));
+  } else {
+    tghi = tb;
+    tglo = tb;
+  }
   Params p{static_cast<int>(Nc), D, r, Dout, top_m, scores, status, wait_limit_ns()};
   SPTS_CUDA_TRY(
       cudaFuncSetAttribute(ltp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM_BYTES)));
-  ltp_kernel<<<static_cast<unsigned>((Nc + 127) / 128), THREADS, SMEM_BYTES, s>>>(tx, ta, tb, p);
+  ltp_kernel<<<static_cast<unsigned>((Nc + 127) / 128), THREADS, SMEM_BYTES, s>>>(tx, ta, tb, tghi, tglo, p);
   note_launch();
   SPTS_CUDA_TRY(cudaGetLastError());
   return SPTS_OK;

@@ -340,4 +340,82 @@ spts_status launch_gather_i32(const int32_t *src, const int32_t *idx, int64_t m,
   return SPTS_OK;
 }
 
+// ---------------------------------------------------------------- bf16 residual boundary
+// dst[i] = float(src[i]) for n elements (n % 8 == 0), 16-byte loads.
+__global__ void bf16_to_f32_kernel(const uint4 *__restrict__ src, int64_t n8, float4 *__restrict__ dst) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const uint4 v = src[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      f[2 * q] = __uint_as_float(w[q] << 16);
+      f[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+    }
+    dst[2 * i] = make_float4(f[0], f[1], f[2], f[3]);
+    dst[2 * i + 1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+}
+
+// dst[rows[t]] = bf16(src[rows[t]]) (round to nearest even) for t < m, rows
+// of D elements (D % 8 == 0): one warp per row, 16-byte stores.
+__global__ void rows_f32_to_bf16_kernel(const float4 *__restrict__ src, const int32_t *__restrict__ rows, int64_t m,
+                                        int64_t n_rows, int d8, uint4 *__restrict__ dst, uint32_t *status) {
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= m) return;
+  const int64_t r = rows[t];
+  if (r < 0 || r >= n_rows) {
+    if (lane == 0) raise_status(status, SPTS_DEV_BADINDEX, 0x61u, static_cast<uint32_t>(r));
+    return;
+  }
+  for (int c = lane; c < d8; c += 32) {
+    const float4 a = src[(r * d8 + c) * 2], b = src[(r * d8 + c) * 2 + 1];
+    dst[r * d8 + c] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                                 pack_bf16x2(b.z, b.w));
+  }
+}
+
+spts_status launch_bf16_to_f32(const void *src, int64_t n, float *dst, cudaStream_t s) {
+  if (n == 0) return SPTS_OK;
+  const int64_t n8 = n / 8;
+  const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, static_cast<int64_t>(num_sms()) * 8);
+  bf16_to_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(static_cast<const uint4 *>(src), n8,
+                                                                      reinterpret_cast<float4 *>(dst));
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+spts_status launch_rows_f32_to_bf16(const float *src, const int32_t *rows, int64_t m, int64_t n_rows, int D,
+                                    void *dst, uint32_t *status, cudaStream_t s) {
+  if (m == 0) return SPTS_OK;
+  rows_f32_to_bf16_kernel<<<static_cast<unsigned>((m + 7) / 8), 256, 0, s>>>(
+      reinterpret_cast<const float4 *>(src), rows, m, n_rows, D / 8, static_cast<uint4 *>(dst), status);
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
+// ---------------------------------------------------------------- test hook
+// y[i] = exp2_poly2(x[i]): the FMA-pipe exp2 of the reduced-attention softmax, on its own.
+__global__ void exp2_poly_kernel(const float *__restrict__ x, int64_t n, float *__restrict__ y) {
+  const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 2;
+  if (i >= n) return;
+  const float a = x[i], b = i + 1 < n ? x[i + 1] : x[i];
+  float e0, e1;
+  exp2_poly2(f2pack(a, b), e0, e1);
+  y[i] = e0;
+  if (i + 1 < n) y[i + 1] = e1;
+}
+
+spts_status launch_exp2_poly(const float *x, int64_t n, float *y, cudaStream_t s) {
+  if (n == 0) return SPTS_OK;
+  exp2_poly_kernel<<<static_cast<unsigned>((n + 511) / 512), 256, 0, s>>>(x, n, y);
+  note_launch();
+  SPTS_CUDA_TRY(cudaGetLastError());
+  return SPTS_OK;
+}
+
 }  // namespace spts

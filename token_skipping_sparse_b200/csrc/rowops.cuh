@@ -55,6 +55,12 @@ spts_status launch_gather_i32(const int32_t *src, const int32_t *idx, int64_t m,
 // device now (CUDA loads a kernel's code lazily, at its first launch or
 // attribute query), so that a later launch takes no device memory for code.
 spts_status preload_gather_rows();
+// bf16 residual boundary: n bf16 -> fp32 (n % 8 == 0); rows[t] of src fp32
+// -> bf16 into dst (D % 8 == 0).
+spts_status launch_bf16_to_f32(const void *src, int64_t n, float *dst, cudaStream_t s);
+spts_status launch_exp2_poly(const float *x, int64_t n, float *y, cudaStream_t s);
+spts_status launch_rows_f32_to_bf16(const float *src, const int32_t *rows, int64_t m, int64_t n_rows, int D,
+                                    void *dst, uint32_t *status, cudaStream_t s);
 spts_status preload_select_topk();
 spts_status launch_iota_i32(int32_t *dst, int64_t n, cudaStream_t s);
 spts_status launch_sum_groups(const float *group, int G, int64_t n, float *s, cudaStream_t st);
@@ -102,8 +108,11 @@ spts_status launch_probe_bf16(const void *q, const int32_t *qpos, int P, const v
 size_t probe_bf16_stats_bytes(int P, int Hq, int64_t Nc);
 
 // top_m > 0 (Dout <= 512): score = sum of the top_m largest |y| instead of ||y||_2.
+// LTP score; top_m == 0 (the L2 norm) needs ltp_gram_bytes(r) of scratch
+// for the Gram matrix in gram_ws, top_m > 0 none.
+size_t ltp_gram_bytes(int r);
 spts_status launch_ltp_bf16(const void *x, int64_t Nc, int D, const void *A, int r, const void *B, int Dout,
-                            float *scores, uint32_t *status, cudaStream_t s, int top_m = 0);
+                            float *scores, uint32_t *status, cudaStream_t s, int top_m, void *gram_ws);
 
 spts_status launch_attention_bf16(const void *q, const int32_t *qpos, int64_t m, const void *k, const void *v,
                                   const int32_t *kpos, int64_t Nc, int Hq, int Hkv, float scale, void *o,

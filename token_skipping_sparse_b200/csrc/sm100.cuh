@@ -434,25 +434,25 @@ __device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
 // 2^x for a pair of x <= 0 on the FMA and integer pipes, leaving the MUFU
 // (exp2) pipe to the other elements of a softmax row.  Range reduction:
 // x = j + f with j = round(x) (adding 1.5 * 2^23 leaves round(x) in the low
-// mantissa bits) and f in [-1/2, 1/2]; 2^f by the degree-3 polynomial of
-// smallest maximum relative error on that interval (7.5e-5; coefficients
-// derived by exp2_poly_fit.py beside this package); j goes into the exponent
-// field by an integer add.  x is clamped at -125 so the exponent stays
-// normal: a masked (-inf) element gives 2^-125 instead of 0, which no bf16
-// probability or fp32 row sum can tell from zero next to the row's maximum
-// (which contributes 1).
+// mantissa bits) and f in [-1/2, 1/2]; 2^f by the degree-3 polynomial with
+// p(0) = 1 of smallest maximum relative error on that interval (1.0e-4;
+// coefficients derived by exp2_poly_fit.py beside this package); j goes into
+// the exponent field by an integer add.  x is clamped at -127: there j = -127
+// and p = 1.0 exactly, whose bits plus -127 in the exponent field are +0, so
+// a masked score (-inf) gives exactly 0.  Below -126 the result is a tiny
+// value (< 2^-125), not 2^x; no softmax row can tell it from 0.
 __device__ __forceinline__ void exp2_poly2(uint64_t x2, float &e0, float &e1) {
   float a, b;
   f2unpack(x2, a, b);
-  const uint64_t x = f2pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t x = f2pack(fmaxf(a, -127.f), fmaxf(b, -127.f));
   const uint64_t shifter = f2pack(12582912.f, 12582912.f);  // 1.5 * 2^23
   const uint64_t y = f2add(x, shifter);
   const uint64_t j = f2add(y, f2pack(-12582912.f, -12582912.f));
   const uint64_t f = f2fma(j, f2pack(-1.f, -1.f), x);
-  uint64_t p = f2fma(f2pack(0.0551716685295105f, 0.0551716685295105f), f,
-                     f2pack(0.2426111251115799f, 0.2426111251115799f));
-  p = f2fma(p, f, f2pack(0.6932609677314758f, 0.6932609677314758f));
-  p = f2fma(p, f, f2pack(0.9999280571937561f, 0.9999280571937561f));
+  uint64_t p = f2fma(f2pack(0.055009059607982635f, 0.055009059607982635f), f,
+                     f2pack(0.2422109693288803f, 0.2422109693288803f));
+  p = f2fma(p, f, f2pack(0.6932829022407532f, 0.6932829022407532f));
+  p = f2fma(p, f, f2pack(1.0f, 1.0f));
   float p0, p1, y0, y1;
   f2unpack(p, p0, p1);
   f2unpack(y, y0, y1);
