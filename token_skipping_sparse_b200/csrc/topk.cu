@@ -5,7 +5,7 @@
 //   2. fused score f per candidate in fp32, one rounding per operation
 //      (w_a*(s/max s) + w_b*(c/max c), or s*c, or s), mapped to an
 //      order-preserving uint32 key (-0 -> +0);
-//   3. MSB-first radix select, 4 digits of 8 bits, over the first Nc - tail
+//   3. MSB-first radix select, digits of 11, 11 and 10 bits, over the first Nc - tail
 //      candidates: finds the key T of the (k - tail)-th largest and how many
 //      keys equal to T must be taken;
 //   4. stable compaction in index order: a candidate is kept if its key > T,
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     select_topk_kernel(FuseArgs fa, int64_t Nc, int64_t k, int64_t tail, int32_t *__restrict__ idx_out,
                        float *__restrict__ fused_out, float *__restrict__ kth_out, uint32_t *status) {
   extern __shared__ uint32_t keys[];  // CACHE: keys of the first Nc - tail candidates
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[2048];
   __shared__ uint32_t warp_tot[32];
   __shared__ float fred[2][32];
   __shared__ uint32_t s_digit, s_krem, s_total;
@@ -180,47 +180,54 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     return order_key(fused(fa, i));
   };
 
-  // 3. radix select of the k_free-th largest key among [0, n_free)
+  // 3. radix select of the k_free-th largest key among [0, n_free): digits of
+  // 11, 11 and 10 bits from the top.  Scores in a narrow range share the
+  // top 8 bits of their keys; taking 3 mantissa bits more into the first
+  // digit spreads them over more bins, so fewer threads collide on one
+  // shared-memory counter.
   uint32_t T = 0xFFFFFFFFu, need_eq = 0;
   if (k_free > 0) {
     uint32_t prefix = 0, mask = 0, krem = static_cast<uint32_t>(k_free);
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int b = tid; b < 256; b += TK_THREADS) hist[b] = 0;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+      const int bits = pass < 2 ? 11 : 10;
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const uint32_t nbins = 1u << bits;
+      for (int b = tid; b < static_cast<int>(nbins); b += TK_THREADS) hist[b] = 0;
       __syncthreads();
       for (int64_t i = tid; i < n_free; i += TK_THREADS) {
         const uint32_t key = key_at(i);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nbins - 1u)], 1u);
       }
       __syncthreads();
       if (w == 0) {
-        // lane l owns bins 255-8l .. 248-8l (descending)
-        uint32_t c[8], sum = 0;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          c[t] = hist[255 - 8 * lane - t];
-          sum += c[t];
-        }
+        // lane l owns the bins nbins-1-l*per .. nbins-(l+1)*per (descending)
+        const int per = static_cast<int>(nbins) >> 5;
+        const int top = static_cast<int>(nbins) - 1 - lane * per;
+        uint32_t sum = 0;  // rotated start per lane: the 32 lanes read 32 different banks
+        for (int t = 0; t < per; ++t) sum += hist[top - (t + lane) % per];
         uint32_t incl = sum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
           if (lane >= o) incl += y;
         }
         uint32_t above = incl - sum;  // keys in bins higher than my first bin
         if (above < krem && krem <= incl) {
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            if (above < krem && krem <= above + c[t]) {
-              s_digit = static_cast<uint32_t>(255 - 8 * lane - t);
+          for (int t = 0; t < per; ++t) {
+            const uint32_t c = hist[top - t];
+            if (above < krem && krem <= above + c) {
+              s_digit = static_cast<uint32_t>(top - t);
               s_krem = krem - above;
+              break;
             }
-            above += c[t];
+            above += c;
           }
         }
       }
       __syncthreads();
       prefix |= s_digit << shift;
-      mask |= 255u << shift;
+      mask |= (nbins - 1u) << shift;
       krem = s_krem;
       __syncthreads();
     }
