@@ -56,6 +56,11 @@ DEFAULT_STEPS = {"attn_8k": 100, "layer_32k": 20, "layer_128k": 10, "msdp_32k": 
                  "llama32": 5}
 
 
+def progress(msg):
+    """One line per phase on stderr (the JSON line stays alone on stdout)."""
+    print(f"bench [{time.strftime('%H:%M:%S')}] {msg}", file=sys.stderr, flush=True)
+
+
 # ---------------------------------------------------------------- peaks
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -254,11 +259,13 @@ def measure_layer(S, wl, args, rank, world, dev, peaks, e2e=True):
             S.spts_layer_forward(h, case.pos, desc, case.weights, events=evs)
             return h
 
+    progress(f"{wl.name}: inputs on the device; {args.warmup} warm-up steps")
     h = (base if msdp else case).h0.clone()
     for _ in range(args.warmup):
         step(h if not msdp else (base.h0.clone()))
     torch.cuda.synchronize()
     S.check_device_status()
+    progress(f"{wl.name}: staged passes")
 
     # ---------------- per-stage breakdown (one layer) and the dominant kernel
     lcase = base if msdp else case
@@ -292,6 +299,7 @@ def measure_layer(S, wl, args, rank, world, dev, peaks, e2e=True):
     torch.cuda.synchronize()
 
     # ---------------- timed region
+    progress(f"{wl.name}: timed region, {args.steps} steps")
     steps = args.steps
     inputs = [base.h0.clone() for _ in range(1)] if msdp else None
     timed_evs = [None] * steps
@@ -347,6 +355,7 @@ def measure_layer(S, wl, args, rank, world, dev, peaks, e2e=True):
               for name, key in (("burst", "bf16"), ("sustained", "bf16_sustained"))}
 
     # ---------------- skipped-prefill speedup over the same kernels at keep 1.0
+    progress(f"{wl.name}: timed {ms_step:.3f} ms per step; keep 1.0 and end to end")
     dense = None
     if not msdp and not args.no_dense:
         ddesc = lcase.desc(k=wl.N)
@@ -471,6 +480,7 @@ def gpu_arm(args, rank, world, dev):
         result["layer_128k"] = sub
     # the 32-layer Table B schedule at 32K (a few prefills): TTFT against keep 1.0
     if args.workload == "layer_32k" and not args.no_schedule:
+        progress("llama32_32k: the 32-layer schedule")
         sargs = argparse.Namespace(**{**vars(args), "workload": "llama32_32k", "steps": 3, "warmup": 1})
         sch = schedule_arm(sargs, rank, world, dev)
         jac = [j["jaccard"] for j in sch["jaccard_consecutive"]]
@@ -485,7 +495,9 @@ def gpu_arm(args, rank, world, dev):
             "clocks": sch["clocks"]}
         torch.cuda.empty_cache()
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        progress("cpu_baseline: one whole layer through the oracle's timed mode")
         result["cpu_baseline"] = cpu_baseline(wl)
+    progress("done")
     return result
 
 
