@@ -9,8 +9,10 @@
 // the tensor core works on the other.
 //   warp 0      TMA: both Q tiles and key tile 0 at entry (while warps 0..3
 //               find the tiles' key ranges by warp-wide searches), then the
-//               other K and V tiles of 128 keys into a 2-stage ring
-//               (128-byte swizzle);
+//               other K and V tiles of 128 keys into two 2-stage rings
+//               (128-byte swizzle); a K stage is released once both tiles'
+//               S MMAs have read it and a V stage once both PVs have, so the
+//               next key tile's load does not wait for the PVs;
 //   warp 1      MMA, per key tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1),
 //               the whole warp running the loop on warp-uniform descriptors
 //               and one elected lane issuing each tcgen05 op (a lone lane
@@ -106,8 +108,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t *sK = smem + OFF_K;
   uint8_t *sV = smem + OFF_V;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-  uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = k_full + KV_STAGES, *kv_empty = v_full + KV_STAGES,
-           *s_full = kv_empty + KV_STAGES, *p_ready = s_full + 2, *o_done = p_ready + 4, *drain = o_done + 2;
+  uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = k_full + KV_STAGES, *k_empty = v_full + KV_STAGES,
+           *v_empty = k_empty + KV_STAGES, *s_full = v_empty + KV_STAGES, *p_ready = s_full + 2,
+           *o_done = p_ready + 4, *drain = o_done + 2;
   // p_ready[2 X + h]: P of tile X for keys [64 h, 64 h + 64) is in TMEM
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -129,7 +132,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int s = 0; s < KV_STAGES; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
@@ -178,19 +182,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_LOW));
     if (lane == 0) {
-      uint32_t issued = 1u, issued_par = 0;  // stage 0: key tile 0, loaded at entry
+      // K and V stages are released separately (K tile j once both tiles'
+      // S(j) have completed, V tile j once both PV(j) have)
+      uint32_t k_issued = 1u, k_par = 0, v_issued = 1u, v_par = 0;  // stage 0: key tile 0, loaded at entry
       for (int j = 1; j < n_kv; ++j) {
         const int st = j % KV_STAGES;
         const uint32_t ph = (j / KV_STAGES) & 1;
-        if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_flag, p.status, p.wait_ns, 0x21u)) break;
+        if (!mbar_wait(&k_empty[st], ph ^ 1u, abort_flag, p.status, p.wait_ns, 0x21u)) break;
         mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
         tma_load_3d(sK + st * TILE_BYTES, &tmK, &k_full[st], 0, g, j * BKV);
         tma_load_3d(sK + st * TILE_BYTES + CHUNK_BYTES, &tmK, &k_full[st], 64, g, j * BKV);
+        k_issued |= 1u << st;
+        k_par = (k_par & ~(1u << st)) | (ph << st);
+        if (!mbar_wait(&v_empty[st], ph ^ 1u, abort_flag, p.status, p.wait_ns, 0x2Au)) break;
         mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
         tma_load_3d(sV + st * TILE_BYTES, &tmV, &v_full[st], 0, g, j * BKV);
         tma_load_3d(sV + st * TILE_BYTES + CHUNK_BYTES, &tmV, &v_full[st], 64, g, j * BKV);
-        issued |= 1u << st;
-        issued_par = (issued_par & ~(1u << st)) | (ph << st);
+        v_issued |= 1u << st;
+        v_par = (v_par & ~(1u << st)) | (ph << st);
       }
       if (n_kv == 0) {  // no visible key: let the entry loads of tile 0 land
         mbar_drain(&k_full[0], 0, p.status);
@@ -198,11 +207,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (*abort_flag) {
         mbar_drain(q_full, 0, p.status);
-        for (int st = 0; st < KV_STAGES; ++st)
-          if (issued & (1u << st)) {
-            mbar_drain(&k_full[st], (issued_par >> st) & 1u, p.status);
-            mbar_drain(&v_full[st], (issued_par >> st) & 1u, p.status);
-          }
+        for (int st = 0; st < KV_STAGES; ++st) {
+          if (k_issued & (1u << st)) mbar_drain(&k_full[st], (k_par >> st) & 1u, p.status);
+          if (v_issued & (1u << st)) mbar_drain(&v_full[st], (v_par >> st) & 1u, p.status);
+        }
       }
     }
     __syncwarp();
@@ -256,6 +264,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       };
       for (int x = 0; ok && x < 2; ++x)
         if ((x == 0 ? n_a : n_b) > 0) ok = issue_s(x, 0);
+      if (ok && n_kv > 0) tc_commit_w(&k_empty[0]);  // both S(0) read key tile 0
       for (int j = 0; ok && j < n_kv; ++j) {
         for (int x = 0; ok && x < 2; ++x) {
           const int nxx = x == 0 ? n_a : n_b;
@@ -263,7 +272,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           ok = issue_pv(x, j);
           if (ok && j + 1 < nxx) ok = issue_s(x, j + 1);
         }
-        if (ok) tc_commit_w(&kv_empty[j % KV_STAGES]);  // both tiles are done with K/V tile j
+        if (!ok) break;
+        // V tile j is free once both PV(j) are done, key tile j + 1 once both
+        // S(j+1) are: the next key tile's load no longer waits for the PVs
+        tc_commit_w(&v_empty[j % KV_STAGES]);
+        if (j + 1 < n_kv) tc_commit_w(&k_empty[(j + 1) % KV_STAGES]);
       }
       tc_commit_w(drain);
       mbar_drain(drain, 0, p.status);
