@@ -124,48 +124,89 @@ def job_throughput(units_per_rank, world, ms_max):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
+    """SM clock and throttle reasons while the timed region runs.
+
+    NVML is polled every 10 ms from a thread (read-only queries), so that a
+    timed region of ~0.1 s still gets about ten samples; where NVML cannot be
+    loaded, nvidia-smi polls every 100 ms instead."""
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    # NVML clock event reason bits, in the order of NAMES
+    BITS = (0x8, 0x40, 0x20, 0x4)
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, dev):
-        self.proc = None
-        self.out = tempfile.TemporaryFile(mode="w+")
+    def __init__(self, dev, period_s=0.01):
+        import threading
+        self.proc = self.thread = None
+        self.samples = []                       # (sm MHz, max MHz, set of reasons)
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
         try:
-            uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.stop_evt = threading.Event()
+
+            def poll():
+                while not self.stop_evt.is_set():
+                    try:
+                        sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                        r = int(reasons(h))
+                        self.samples.append((sm, mx, {n for n, b in zip(self.NAMES, self.BITS) if r & b}))
+                    except Exception:
+                        pass
+                    self.stop_evt.wait(period_s)
+
+            self.source = f"NVML every {int(period_s * 1000)} ms"
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
+        self.out = tempfile.TemporaryFile(mode="w+")
+        self.source = "nvidia-smi every 100 ms"
+        try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.out, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return None
+    def _smi_samples(self):
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.out.seek(0)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.out.read().splitlines():
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 7:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
+                sm, mx = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+            self.samples.append((sm, mx, {n for n, v in zip(self.NAMES, parts[3:7])
+                                          if v.lower().startswith("active")}))
+
+    def stop(self):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+        elif self.proc is not None:
+            self._smi_samples()
+        else:
+            return None
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        reasons = set().union(*(r for _, _, r in self.samples))
+        return {"sm_mhz": statistics.median(s for s, _, _ in self.samples),
+                "sm_max_mhz": max(m for _, m, _ in self.samples), "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": self.source}
 
 
 # ---------------------------------------------------------------- the GPU arm
@@ -385,11 +426,13 @@ def measure_layer(S, wl, args, rank, world, dev, peaks, e2e=True):
             # directions at once).  Every step moves its own input in and its
             # result out.  io_bf16: the residual crosses the boundary in bf16
             # (spts_layer_forward_bf16io), else in fp32 (spts_layer_forward).
+            # The timed region covers the same K steps as the device timing,
+            # from the first step's H2D to the last step's D2H.
             dt = torch.bfloat16 if io_bf16 else torch.float32
             hh = lcase.h0.to(dt).cpu().pin_memory()
             ho = torch.empty_like(hh).pin_memory()
             NBUF = 3
-            ne = min(steps, 10)
+            ne = steps
             dbuf = [torch.empty_like(lcase.h0, dtype=dt) for _ in range(NBUF)]
             s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
             ev_in = [torch.cuda.Event() for _ in range(NBUF)]
