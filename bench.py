@@ -557,7 +557,7 @@ def timed_case(wl):
 
 
 def timed_supported(wl):
-    return (wl.F > 0 and not wl.kv_active and not wl.ltp_top_m and not wl.ltp_dout
+    return (not wl.kv_active and not wl.ltp_top_m and not wl.ltp_dout
             and wl.fuse in (FUSE_NONE, FUSE_MAXNORM_ADD, FUSE_MULTIPLY))
 
 
@@ -566,7 +566,8 @@ def time_oracle_layer(wl, case):
     from oracle import timed as T
     k, h, W, sal, pos = case
     t0 = time.perf_counter()
-    T.layer_forward(h, pos, W, wl.Hq, wl.Hkv, wl.P, k, wl.fuse, salient_rows=sal, salient_shift=wl.salient_shift)
+    T.layer_forward(h, pos, W, wl.Hq, wl.Hkv, wl.P, k, wl.fuse, salient_rows=sal, salient_shift=wl.salient_shift,
+                    ffn=wl.F > 0)
     return time.perf_counter() - t0
 
 
@@ -575,11 +576,13 @@ def cpu_baseline(wl):
     (every row, every step of the layer), measured, not scaled."""
     if not timed_supported(wl):
         return {"kind": "oracle", "unavailable": f"{wl.name}: the oracle's timed mode covers the MaxNorm-Add / "
-                                                 "Multiply layers with the L2 proxy score and all-candidate keys"}
+                                                 "Multiply layers (and the attention-only layer) with the L2 "
+                                                 "proxy score and all-candidate keys"}
     case = timed_case(wl)
     dt = time_oracle_layer(wl, case)
     threads = torch.get_num_threads()
-    what = "the first layer of MSDP stage 1" if wl.ratios else "one whole layer"
+    what = ("the first layer of MSDP stage 1" if wl.ratios else
+            "one attention-only layer (no FFN)" if wl.F == 0 else "one whole layer")
     return {"value": round(wl.N / dt, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{wl.name}: {what} (N = {wl.N} rows, k = {case[0]}), every step in full, through the "
                       f"oracle's fp32 timed mode (oracle/timed.py: plain torch CPU ops) on {threads} host threads; "
@@ -777,7 +780,8 @@ def reference_arm(args):
     ms = 1000.0 * wall / args.steps
     v = round(wl.N / (ms / 1000.0), 2)
     threads = torch.get_num_threads()
-    what = "the first layer of MSDP stage 1" if wl.ratios else "one whole layer"
+    what = ("the first layer of MSDP stage 1" if wl.ratios else
+            "one attention-only layer (no FFN)" if wl.F == 0 else "one whole layer")
     cb = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
           "sample": f"{wl.name}: {what} per step (N = {wl.N}, k = {case[0]}), every step of the layer in full, "
                     f"through the oracle's fp32 timed mode on {threads} host threads; not scaled",

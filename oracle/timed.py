@@ -87,10 +87,11 @@ def _attention(q, q_pos, kk, vv, key_pos, G, slab=1024):
 
 
 def layer_forward(h, pos, W, Hq, Hkv, P, k, fuse=FUSE_MAXNORM_ADD, w_a=0.5, w_b=0.5, salient_rows=None,
-                  salient_shift=0.0):
+                  salient_shift=0.0, ffn=True):
     """One SPTS layer in fp32 on the host: h [Nc, D] fp32 (updated copy
     returned), pos [Nc] int64 ascending, W a dict of fp32 weights (nn.Linear
-    layout; norm weights taken as ones).  Returns (h_out, s, c, f, idx_attn, idx_ffn)."""
+    layout; norm weights taken as ones).  Returns (h_out, s, c, f, idx_attn, idx_ffn);
+    ffn=False is the attention-only layer (steps a1..a7: c, f and idx_ffn None)."""
     Nc, D = h.shape
     d = W["w_q"].shape[0] // Hq
     G = Hq // Hkv
@@ -113,6 +114,8 @@ def layer_forward(h, pos, W, Hq, Hkv, P, k, fuse=FUSE_MAXNORM_ADD, w_a=0.5, w_b=
     o_sel = _bf16(_attention(q_sel, pos[idx_a], kk, vv, pos, G))
     h1 = h.clone()
     h1[idx_a] += o_sel.view(k, Hq * d) @ W["w_o"].T
+    if not ffn:
+        return h1, s, None, None, idx_a, None
     # LTP score of the FFN input (Fig. 2(b)): || (x A^T) B^T ||_2
     x2 = _bf16(_rmsnorm(h1))
     c = (_bf16(x2 @ W["ltp_a"].T) @ W["ltp_b"].T).norm(dim=1)

@@ -37,6 +37,31 @@ def test_reduced_attention_bf16(Nc, k, Hq, Hkv):
     assert np.mean(np.abs(got - want)) < 2e-3
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (8, 4), (32, 8)])
+def test_reduced_attention_bf16_lopsided_tile_pairs(Hq, Hkv):
+    """A CTA's two Q tiles with very different key ranges: the first tile of
+    each pair sees one or two key tiles, the second dozens, so for most key
+    steps only the second tile runs and the K and V stages are recycled by
+    its MMAs alone; the last pair is a single partial tile."""
+    Nc, tq = 4096, 128 // (Hq // Hkv)
+    pos = np.arange(Nc, dtype=np.int32) * 2 + 1
+    early = np.arange(tq)                              # keys 0 .. tq-1
+    late = np.arange(Nc - 40 * tq, Nc - 39 * tq)       # most of the keys
+    tail = np.arange(Nc - 3 * tq // 2, Nc)             # last pair: one full tile and half of the next
+    sel = np.concatenate([early, late, np.arange(Nc - 38 * tq, Nc - 36 * tq), tail]).astype(np.int64)
+    assert np.all(np.diff(sel) > 0)
+    k = len(sel)
+    q = torch.randn(k, Hq, 128).to(torch.bfloat16)
+    kk = torch.randn(Nc, Hkv, 128).to(torch.bfloat16)
+    v = torch.randn(Nc, Hkv, 128).to(torch.bfloat16)
+    o = S.spts_reduced_attention(q.cuda(), torch.from_numpy(pos[sel]).cuda(), kk.cuda(), v.cuda(),
+                                 torch.from_numpy(pos).cuda())
+    want = O.reduced_attention(np64(q), pos[sel], np64(kk), np64(v), pos)
+    got = np64(o)
+    assert_close(got, want, 2e-2, "reduced attention bf16, lopsided pairs")
+    assert np.mean(np.abs(got - want)) < 2e-3
+
+
 @pytest.mark.parametrize("Nc,P,Hq,Hkv", [(1000, 16, 8, 2), (3000, 64, 32, 8), (2000, 128, 32, 8), (300, 64, 8, 8),
                                          (700, 20, 8, 4), (2500, 80, 32, 8), (130, 100, 32, 8), (1000, 1, 32, 8)])
 def test_probe_scores_bf16(Nc, P, Hq, Hkv):

@@ -46,6 +46,30 @@ def test_timed_layer_matches_fp64_oracle(name):
     assert np.abs(ho.double().numpy() - tr["h_out"]).max() <= 2e-2
 
 
+def test_timed_attention_only_layer_matches_fp64_oracle():
+    """The attention-only layer (the 8K configuration's steps): h after the
+    O projection, the probe scores and the MHA selection."""
+    wl = WORKLOADS["layer_small"]
+    h = make_hidden(wl)
+    W = make_layer_weights(wl)
+    sal = salient_rows(wl.N, wl.P, wl.salient_frac, wl.seed)
+    pos = torch.arange(wl.N)
+    ho, s, c, f, ia, idf = T.layer_forward(h, pos, {n: t.float() for n, t in W.items()}, wl.Hq, wl.Hkv, wl.P, wl.k,
+                                           wl.fuse, salient_rows=sal.long(), salient_shift=wl.salient_shift,
+                                           ffn=False)
+    assert c is None and f is None and idf is None
+    cfg = O.LayerConfig(Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, P=wl.P, k=wl.k, fuse=wl.fuse, salient_rows=sal.numpy(),
+                        salient_shift=wl.salient_shift, ffn=False)
+    tr = {}
+    want, _ = O.layer_forward(h.double().numpy(), pos.numpy(), O.LayerWeights(**_f64(W)), cfg, tr)
+    assert np.abs(s.numpy() - tr["s"]).max() <= 1e-4 * tr["s"].max()
+    assert np.array_equal(ia.numpy(), tr["idx_attn"])
+    assert np.abs(ho.double().numpy() - tr["h_attn"]).max() <= 2e-2
+    assert np.abs(ho.double().numpy() - want).max() <= 2e-2
+    rest = np.setdiff1d(np.arange(wl.N), ia.numpy())
+    assert torch.equal(ho[rest], h[rest])
+
+
 def test_timed_attention_key_range_is_exact():
     """Each slab reads keys up to its last query's position only: the same
     result as masked attention over every key (brute force, fp64 oracle)."""
