@@ -762,6 +762,50 @@ def attention_arm(args, rank, world, dev):
                          "frac": round(ach / peaks["bf16"], 4), "traffic": None}}
 
 
+def topk_arm(args, rank, world, dev):
+    """spts_select_topk alone on a workload's candidate count: the FFN-set
+    selection of the layer (MaxNorm-Add fusion of two seeded positive score
+    vectors, k of them kept with the last P forced, the fused scores written
+    out).  Up to 20K free candidates one CTA runs it, above that the grid
+    path.  The calls are queued behind a sleep kernel so that the timed
+    region holds their device time back to back, not the host's time to
+    issue them (a few microseconds of kernels per call)."""
+    import token_skipping_sparse_b200 as S
+    wl = WORKLOADS[args.workload]
+    peaks = measured_peaks()
+    g = torch.Generator().manual_seed(wl.seed + 12)
+    N, k = wl.N, wl.k
+    s_a = -torch.log1p(-torch.rand(N, generator=g)) * (wl.P * wl.Hq / N)   # sums to about P·Hq, like PAP scores
+    s_b = 26.0 + 2.0 * torch.randn(N, generator=g)                           # LTP row norms at these inits
+    s_a, s_b = s_a.float().to(dev), s_b.abs().float().to(dev)
+    ws = S.workspace(int(S.lib.spts_select_topk_workspace(N)))
+    call = lambda: S.spts_select_topk(s_a, k, wl.P, s_b=s_b, mode=FUSE_MAXNORM_ADD, fused=True, ws=ws)  # noqa: E731
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    S.check_device_status()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(20_000_000)       # ~10 ms of device time while the calls are queued behind it
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    nbytes = 3 * N * 4 + k * 4           # two score vectors read, the fused scores and k indices written
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"metric": "top-k selection time (kernel alone)", "value": round(ms * 1e3, 2), "unit": "us",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded exponential and |N(26, 2)| score vectors)",
+            "config": {"workload": wl.name, "kernel": "select_topk", "Nc": N, "k": k, "force_tail": wl.P,
+                       "fuse": "maxnorm_add", "path": "grid" if N - wl.P > 20480 else "one CTA"},
+            "roofline": {"bound": "latency", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 5), "traffic": None,
+                         "note": f"{nbytes / 1e6:.2f} MB per call: far below what HBM time would matter for; the "
+                                 "call is bound by its passes' latency (launches, block-wide scans)"}}
+
+
 def reference_arm(args):
     """The oracle (fp32 timed mode) on the host cores: one whole layer per
     step, on the GPU arm's workload, config, metric and unit."""
@@ -805,7 +849,7 @@ def main():
     ap.add_argument("--no-128k", action="store_true", help="time only the 32K layer in the default line")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) measurement")
     ap.add_argument("--no-schedule", action="store_true", help="leave the 32-layer schedule out of the default line")
-    ap.add_argument("--kernel", default=None, choices=["attention"],
+    ap.add_argument("--kernel", default=None, choices=["attention", "topk"],
                     help="time one kernel alone on the workload's shapes (for profiling)")
     args = ap.parse_args()
     if args.steps is None:
@@ -829,6 +873,8 @@ def main():
     try:
         if args.kernel == "attention":
             res = attention_arm(args, rank, world, dev)
+        elif args.kernel == "topk":
+            res = topk_arm(args, rank, world, dev)
         elif WORKLOADS[args.workload].schedule:
             res = schedule_arm(args, rank, world, dev)
         else:

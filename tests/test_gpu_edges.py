@@ -25,9 +25,10 @@ def test_select_all_equal_scores_takes_lowest_indices():
 
 
 
-@pytest.mark.parametrize("Nc,k,tail", [(100000, 20000, 128), (70000, 70000, 64), (70000, 64, 64), (50000, 1, 0)])
+@pytest.mark.parametrize("Nc,k,tail", [(100000, 20000, 128), (70000, 70000, 64), (70000, 64, 64), (50000, 1, 0),
+                                       (30000, 9000, 64)])
 def test_select_large_sets_on_the_grid_path(Nc, k, tail):
-    # above 48K free candidates the selection runs on the grid; all-equal
+    # above 20K free candidates the selection runs on the grid; all-equal
     # scores put every key in one radix bin, few distinct values make long
     # runs of ties at the threshold
     for s in (np.full(Nc, 0.125, np.float32), rng.integers(0, 5, Nc).astype(np.float32) * 0.5):

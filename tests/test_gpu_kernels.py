@@ -117,7 +117,8 @@ def test_gather_rows_and_bad_index():
 
 
 # ---------------------------------------------------------------- selection
-@pytest.mark.parametrize("Nc,k,tail", [(1000, 300, 16), (1000, 1000, 16), (1000, 16, 16), (49280, 9830, 64),
+@pytest.mark.parametrize("Nc,k,tail", [(1000, 300, 16), (1000, 1000, 16), (1000, 16, 16), (20544, 6163, 64),
+                                       (20545, 6163, 64), (32768, 9830, 64), (49280, 9830, 64),
                                        (60000, 12000, 128), (131072, 26214, 128), (7, 3, 0), (1, 1, 1)])
 @pytest.mark.parametrize("mode", [0, 1, 2, 3])
 def test_select_topk_bit_exact(Nc, k, tail, mode):

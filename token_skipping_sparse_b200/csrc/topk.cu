@@ -24,11 +24,11 @@ constexpr int TK_THREADS = 1024;
 constexpr int TK_ITEMS = 8;
 constexpr int TK_SMEM_KEYS = 49152;  // 192 KB of cached keys
 // Above this many free candidates the grid path runs (given scratch).
-// Measured inside the 32K layer: one CTA 34 / 66 us for the two selections,
-// the grid 42 / 82 us (its five launches cost more than they save there);
-// at 128K one CTA 147-316 us against 53-60 us for the grid.
+// Measured alone (MaxNorm-Add, keep 0.3): the grid path takes ~30 us from
+// 26K to 131K candidates, one CTA 25 us at 16K, 35 us at 26K, 39 us at 32K
+// and 53 us at 48K.
 #ifndef TK_GRID_MIN
-#define TK_GRID_MIN 49152
+#define TK_GRID_MIN 20480
 #endif
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -287,11 +287,16 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 //   topk_keys_kernel      (grid)   maxima of the block maxima, fused score,
 //                                  key per candidate into the scratch buffer,
 //                                  histogram of the top 11 key bits;
-//   topk_threshold_kernel (1 CTA)  the bin of the (k - tail)-th largest key,
-//                                  then two more radix digits (11 + 10 bits)
-//                                  over the keys: the threshold T and how
-//                                  many keys equal to T are taken;
-//   topk_count_kernel     (grid)   per chunk, the keys > T and == T;
+//   topk_digit_kernel     (grid, twice)  every CTA finds the bin of the
+//                                  (k - tail)-th largest key in the digits
+//                                  so far (a block scan of each histogram),
+//                                  then histograms the next digit (bits
+//                                  [20, 10), then [9, 0)) of its chunk's keys
+//                                  that share that prefix;
+//   topk_count_kernel     (grid)   the threshold T from the three digits and
+//                                  how many keys equal to T are taken (CTA 0
+//                                  records them), then per chunk the keys > T
+//                                  and == T;
 //   topk_write_kernel     (grid)   the counts of the chunks before its own,
 //                                  then stable compaction of its chunk; CTA 0
 //                                  appends the forced tail.
@@ -300,11 +305,10 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 constexpr int TG_THREADS = 1024;
 constexpr int TG_MAX_CTAS = 256;
 constexpr int TG_BINS = 2048;
-constexpr int TG_LOADS = 8;
 
 struct TopkScratch {
   uint32_t *keys;     // [n_free]
-  uint32_t *hist;     // [TG_BINS]
+  uint32_t *hist;     // [3][TG_BINS]: the histograms of the three digits
   float *maxpart;     // [2][TG_MAX_CTAS]
   double *sumpart;    // [4][TG_MAX_CTAS]: sums of s, s^2, c, c^2 (STD_ADD)
   uint32_t *chunk;    // [2][TG_MAX_CTAS]: per chunk, keys > T and keys == T
@@ -319,7 +323,7 @@ __host__ __device__ inline TopkScratch tg_carve(void *base, int64_t n_free) {
   t.keys = reinterpret_cast<uint32_t *>(p);
   p += tg_round(static_cast<size_t>(n_free) * 4);
   t.hist = reinterpret_cast<uint32_t *>(p);
-  p += tg_round(TG_BINS * 4);
+  p += tg_round(3 * TG_BINS * 4);
   t.maxpart = reinterpret_cast<float *>(p);
   p += tg_round(2 * TG_MAX_CTAS * 4);
   t.sumpart = reinterpret_cast<double *>(p);
@@ -334,7 +338,7 @@ __global__ void __launch_bounds__(TG_THREADS)
     topk_prep_kernel(FuseArgs fa, int64_t Nc, int64_t chunk, TopkScratch t) {
   __shared__ float red[2][32];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  for (int b = blockIdx.x * TG_THREADS + tid; b < TG_BINS; b += gridDim.x * TG_THREADS) t.hist[b] = 0u;
+  for (int b = blockIdx.x * TG_THREADS + tid; b < 3 * TG_BINS; b += gridDim.x * TG_THREADS) t.hist[b] = 0u;
   const int64_t i0 = blockIdx.x * chunk, i1 = min(Nc, i0 + chunk);
   if (fa.mode == SPTS_FUSE_STD_ADD) {
     __shared__ double dred[4][32];
@@ -471,58 +475,71 @@ __device__ __forceinline__ void tg_find_bin(const uint32_t *h, int nb, uint32_t 
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(TG_THREADS, 1)
-    topk_threshold_kernel(int64_t n_free, int64_t k_free, TopkScratch t, float *__restrict__ kth_out) {
+// The first `ndig` digits (11, 11, 10 bits from the top) of the key of the
+// k_free-th largest key, from the histograms in t.hist: prefix and mask of
+// those bits and the rank of that key among the keys sharing the prefix.
+// Every thread of the CTA gets the same values.
+__device__ __forceinline__ void tg_pick(const TopkScratch &t, int ndig, uint32_t k_free, uint32_t *h,
+                                        uint32_t *warp_tot, uint32_t *s_total, uint32_t *s_digit, uint32_t *s_krem,
+                                        uint32_t &prefix, uint32_t &mask, uint32_t &krem) {
+  prefix = 0u;
+  mask = 0u;
+  krem = k_free;
+  for (int d = 0; d < ndig; ++d) {
+    const int shift = d == 0 ? 21 : d == 1 ? 10 : 0;
+    const int nb = d == 2 ? 1024 : 2048;
+    for (int b = threadIdx.x; b < nb; b += TG_THREADS) h[b] = __ldcg(t.hist + d * TG_BINS + b);
+    __syncthreads();
+    tg_find_bin(h, nb, krem, warp_tot, s_total, s_digit, s_krem);
+    prefix |= *s_digit << shift;
+    mask |= static_cast<uint32_t>(nb - 1) << shift;
+    krem = *s_krem;
+    __syncthreads();  // h and the shared results are reused
+  }
+}
+
+// Digit `dig` (1: bits [20, 10), 2: bits [9, 0)) of the chunk's keys that
+// share the threshold's first `dig` digits, added into t.hist[dig].
+__global__ void __launch_bounds__(TG_THREADS)
+    topk_digit_kernel(int64_t n_free, int64_t k_free, int64_t chunk2, int dig, TopkScratch t) {
   __shared__ uint32_t h[TG_BINS];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t s_total, s_digit, s_krem;
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  uint32_t T = 0xFFFFFFFFu, need_eq = 0u;
-  if (k_free > 0) {
-    for (int b = tid; b < TG_BINS; b += TG_THREADS) h[b] = t.hist[b];
-    __syncthreads();
-    tg_find_bin(h, TG_BINS, static_cast<uint32_t>(k_free), warp_tot, &s_total, &s_digit, &s_krem);
-    uint32_t prefix = s_digit << 21, mask = 0x7FFu << 21, krem = s_krem;
-    // two more digits: bits [20, 10) and [9, 0)
-    for (int d = 0; d < 2; ++d) {
-      const int shift = d == 0 ? 10 : 0;
-      const int nb = d == 0 ? 2048 : 1024;
-      for (int b = tid; b < TG_BINS; b += TG_THREADS) h[b] = 0u;
-      __syncthreads();
-      // eight loads in flight per thread: one CTA streams all keys from L2
-      for (int64_t base = 0; base < n_free; base += TG_THREADS * TG_LOADS) {
-        uint32_t kv[TG_LOADS];
-#pragma unroll
-        for (int q = 0; q < TG_LOADS; ++q) {
-          const int64_t i = base + q * TG_THREADS + tid;
-          kv[q] = i < n_free ? __ldcg(t.keys + i) : ~prefix;  // ~prefix never matches
-        }
-#pragma unroll
-        for (int q = 0; q < TG_LOADS; ++q)
-          warp_hist_add(h, (kv[q] >> shift) & static_cast<uint32_t>(nb - 1), (kv[q] & mask) == prefix);
-      }
-      __syncthreads();
-      tg_find_bin(h, nb, krem, warp_tot, &s_total, &s_digit, &s_krem);
-      prefix |= s_digit << shift;
-      mask |= static_cast<uint32_t>(nb - 1) << shift;
-      krem = s_krem;
-    }
-    T = prefix;
-    need_eq = krem;
+  uint32_t prefix, mask, krem;
+  tg_pick(t, dig, static_cast<uint32_t>(k_free), h, warp_tot, &s_total, &s_digit, &s_krem, prefix, mask, krem);
+  const int shift = dig == 1 ? 10 : 0;
+  const uint32_t nb = dig == 1 ? 2048u : 1024u;
+  for (int b = threadIdx.x; b < TG_BINS; b += TG_THREADS) h[b] = 0u;
+  __syncthreads();
+  const int64_t i0 = blockIdx.x * chunk2, i1 = min(n_free, i0 + chunk2);
+  for (int64_t base = i0; base < i1; base += TG_THREADS) {
+    const int64_t i = base + threadIdx.x;
+    const uint32_t key = i < i1 ? __ldcg(t.keys + i) : 0u;
+    warp_hist_add(h, (key >> shift) & (nb - 1u), i < i1 && (key & mask) == prefix);
   }
-  if (tid == 0) {
-    t.sel[0] = T;
-    t.sel[1] = need_eq;
-    if (kth_out) *kth_out = k_free > 0 ? key_value(T) : __uint_as_float(0x7FC00000u);
-  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < static_cast<int>(nb); b += TG_THREADS)
+    if (h[b]) atomicAdd(&t.hist[dig * TG_BINS + b], h[b]);
 }
 
 // Per chunk: keys > T and == T (chunk c = keys [c chunk2, (c + 1) chunk2)).
 __global__ void __launch_bounds__(TG_THREADS)
-    topk_count_kernel(int64_t n_free, int64_t chunk2, TopkScratch t) {
+    topk_count_kernel(int64_t n_free, int64_t k_free, int64_t chunk2, TopkScratch t, float *__restrict__ kth_out) {
   __shared__ uint32_t red[2][32];
+  __shared__ uint32_t h[TG_BINS];
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t s_total, s_digit, s_krem;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const uint32_t T = t.sel[0];
+  uint32_t T = 0xFFFFFFFFu, need_eq = 0u;  // no free pick: no key is above or at T
+  if (k_free > 0) {
+    uint32_t mask;
+    tg_pick(t, 3, static_cast<uint32_t>(k_free), h, warp_tot, &s_total, &s_digit, &s_krem, T, mask, need_eq);
+  }
+  if (blockIdx.x == 0 && tid == 0) {
+    t.sel[0] = T;
+    t.sel[1] = need_eq;
+    if (kth_out) *kth_out = k_free > 0 ? key_value(T) : __uint_as_float(0x7FC00000u);
+  }
   const int64_t i0 = blockIdx.x * chunk2, i1 = min(n_free, i0 + chunk2);
   uint32_t gt = 0, eq = 0;
   for (int64_t i = i0 + tid; i < i1; i += TG_THREADS) {
@@ -618,7 +635,7 @@ __global__ void __launch_bounds__(TG_THREADS)
 }
 
 size_t topk_scratch_bytes(int64_t Nc) {
-  return tg_round(static_cast<size_t>(Nc > 0 ? Nc : 1) * 4) + tg_round(TG_BINS * 4) + tg_round(2 * TG_MAX_CTAS * 4) +
+  return tg_round(static_cast<size_t>(Nc > 0 ? Nc : 1) * 4) + tg_round(3 * TG_BINS * 4) + tg_round(2 * TG_MAX_CTAS * 4) +
          tg_round(4 * TG_MAX_CTAS * 8) + tg_round(4 * TG_MAX_CTAS * 4) + 256;
 }
 
@@ -637,12 +654,13 @@ spts_status launch_select_topk(const float *s_a, const float *s_b, int mode, flo
     note_launch();
     topk_keys_kernel<<<n_cta, TG_THREADS, 0, s>>>(fa, Nc, n_free, chunk, n_cta, t, fused_out, status);
     note_launch();
-    topk_threshold_kernel<<<1, TG_THREADS, 0, s>>>(n_free, k - force_tail, t, kth_out);
+    if (k > force_tail)
+      for (int dig = 1; dig <= 2; ++dig) {
+        topk_digit_kernel<<<n_cta, TG_THREADS, 0, s>>>(n_free, k - force_tail, chunk2, dig, t);
+        note_launch();
+      }
+    topk_count_kernel<<<n_cta, TG_THREADS, 0, s>>>(n_free, k - force_tail, chunk2, t, kth_out);
     note_launch();
-    if (k > force_tail) {
-      topk_count_kernel<<<n_cta, TG_THREADS, 0, s>>>(n_free, chunk2, t);
-      note_launch();
-    }
     topk_write_kernel<<<n_cta, TG_THREADS, 0, s>>>(n_free, k - force_tail, force_tail, chunk2, t, idx_out);
     note_launch();
     SPTS_CUDA_TRY(cudaGetLastError());
