@@ -42,6 +42,47 @@ def test_linear_store_more_tiles_than_sm_pairs():
     assert_bf16_close(np64(out), want, 1e-4, "linear store, many tiles")
 
 
+@pytest.mark.parametrize("epi", ["store", "rope", "swiglu", "scatter"])
+def test_linear_whole_round_then_half_tiles(epi):
+    # 10 x 8 = 80 two-SM tiles over 74 resident CTA pairs on a B200: one round
+    # of whole 256 x 256 tiles, then the 6 tiles left run as 12 halves of 128
+    # columns (N = 128 MMAs); M is ragged
+    M, K, N = 2500, 128, 2048
+    A = torch.randn(M, K).to(torch.bfloat16)
+    Ad = A.cuda()
+    if epi == "store":
+        W = _w(N, K)
+        got = np64(S.spts_linear(Ad, W.cuda()))
+        want = O.bf16_round(np64(A) @ np64(W).T)
+    elif epi == "rope":
+        W = _w(N, K)
+        pos = torch.from_numpy(np.sort(rng.choice(200000, M, replace=False)).astype(np.int32))
+        got = np64(S.spts_linear(Ad, W.cuda(), S.EPI_ROPE, row_pos=pos.cuda(), theta=500000.0))
+        want = O.bf16_round(O.rope((np64(A) @ np64(W).T).reshape(M, N // 128, 128), pos.numpy(),
+                                   500000.0)).reshape(M, -1)
+    elif epi == "swiglu":
+        F = N // 2                                     # 8 tiles of 128 gate + 128 up columns
+        Wg, Wu = _w(F, K, 0.1), _w(F, K, 0.1)
+        got = np64(S.spts_linear(Ad, Wg.cuda(), S.EPI_SWIGLU, W2=Wu.cuda()))
+        g, u = np64(A) @ np64(Wg).T, np64(A) @ np64(Wu).T
+        want = O.bf16_round(g / (1 + np.exp(-g)) * u)
+    else:
+        W = _w(N, K)
+        Nc = 3000
+        h = torch.randn(Nc, N)
+        rows = torch.from_numpy(rng.choice(Nc, M, replace=False).astype(np.int32))
+        hd = h.cuda()
+        S.spts_linear(Ad, W.cuda(), S.EPI_SCATTER_ADD, out=hd, rows=rows.cuda())
+        want = np64(h)
+        want[rows.numpy()] += np64(A) @ np64(W).T
+        got = np64(hd)
+        skip = np.setdiff1d(np.arange(Nc), rows.numpy())
+        assert np.array_equal(got[skip], np64(h)[skip])
+        assert_close(got, want, 1e-4, "scatter add, halves")
+        return
+    assert_bf16_close(got, want, 1e-4, f"linear {epi}, halves")
+
+
 @pytest.mark.parametrize("lo,hi", [(0, 200000), (2 ** 24 - 170, 2 ** 24 + 163), (2 ** 30, 2 ** 31 - 1)])
 def test_linear_rope(lo, hi):
     # positions below 2^24 take the fp32 two-product angle reduction, from

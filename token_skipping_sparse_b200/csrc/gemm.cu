@@ -42,6 +42,7 @@ constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + STG_BYTES;
 struct Params {
   int M, N, K;         // N: output columns of W (for SWIGLU: of W_gate and of W_up each)
   int tiles_m, tiles_n;
+  int split_from;      // two-SM tiles from this index on run as two 128-column halves
   void *out;
   const int32_t *rows;
   const int32_t *row_pos;
@@ -76,20 +77,21 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float *v
 }
 
 
-// Fused epilogue of one 256-column accumulator tile for the 32 rows this warp
-// owns: `tbase` addresses the warp's TMEM lanes at the tile's first column;
-// `row` is this thread's output row, `tn` the tile's column index.
+// Fused epilogue of one accumulator tile of `width` columns (256, or 128
+// for half a tile) for the 32 rows this warp owns: `tbase` addresses the
+// warp's TMEM lanes at the tile's first column; `row` is this thread's
+// output row, `col0` the output column of the tile's first result column.
 template <int EPI>
-__device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, int64_t row, bool live, int tn,
-                                              float *stg) {
+__device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, int64_t row, bool live, int col0,
+                                              int width, float *stg) {
   if (EPI == SPTS_EPI_STORE) {
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = 0; c < width / 32; ++c) {
       uint32_t r[32];
       tmem_ld32(tbase + c * 32, r);
       tmem_ld_wait();
-      if (live) store_bf16x32(out + row * p.N + tn * BN + c * 32, reinterpret_cast<float *>(r));
+      if (live) store_bf16x32(out + row * p.N + col0 + c * 32, reinterpret_cast<float *>(r));
     }
   } else if (EPI == SPTS_EPI_ROPE) {
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
@@ -101,7 +103,7 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
 #pragma unroll
       for (int i = 0; i < 32; ++i) rope_cos_sin(pos, p.freqs, c * 32 + i, &cs[i], &sn[i]);
 #pragma unroll 1
-      for (int hc = 0; hc < BN / 128; ++hc) {   // heads of 128 columns in this tile
+      for (int hc = 0; hc < width / 128; ++hc) {   // heads of 128 columns in this tile
         uint32_t lo[32], hi[32];
         tmem_ld32(tbase + hc * 128 + c * 32, lo);
         tmem_ld32(tbase + hc * 128 + 64 + c * 32, hi);
@@ -114,7 +116,7 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
           yh[i] = xh * cs[i] + xl * sn[i];
         }
         if (live) {
-          __nv_bfloat16 *o = out + row * p.N + tn * BN + hc * 128;
+          __nv_bfloat16 *o = out + row * p.N + col0 + hc * 128;
           store_bf16x32(o + c * 32, yl);
           store_bf16x32(o + 64 + c * 32, yh);
         }
@@ -123,15 +125,15 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
   } else if (EPI == SPTS_EPI_SWIGLU) {
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < width / 64; ++c) {      // gate in the first half of the columns, up in the second
       uint32_t g[32], u[32];
       tmem_ld32(tbase + c * 32, g);
-      tmem_ld32(tbase + 128 + c * 32, u);
+      tmem_ld32(tbase + width / 2 + c * 32, u);
       tmem_ld_wait();
       float y[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) y[i] = silu(__uint_as_float(g[i])) * __uint_as_float(u[i]);
-      if (live) store_bf16x32(out + row * p.N + tn * 128 + c * 32, y);
+      if (live) store_bf16x32(out + row * p.N + col0 + c * 32, y);
     }
   } else {  // SCATTER_ADD into fp32 rows (unique rows): each 32-column chunk of the warp's 32 rows goes
            // through shared memory so that 8 lanes update one row's 128 contiguous bytes: coalesced
@@ -144,7 +146,7 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
     for (int i = 0; i < 8; ++i) dst[i] = __shfl_sync(0xffffffffu, orow, 4 * i + (lane >> 3));
     float4 *srow = reinterpret_cast<float4 *>(stg + lane * STG_STRIDE);
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = 0; c < width / 32; ++c) {
       uint32_t r[32];
       tmem_ld32(tbase + c * 32, r);
       tmem_ld_wait();
@@ -157,7 +159,7 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         if (dst[i] >= 0)
-          hv[i] = reinterpret_cast<const float4 *>(out + dst[i] * p.N + tn * BN + c * 32)[lane & 7];
+          hv[i] = reinterpret_cast<const float4 *>(out + dst[i] * p.N + col0 + c * 32)[lane & 7];
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         if (dst[i] >= 0) {
@@ -166,7 +168,7 @@ __device__ __forceinline__ void epilogue_rows(const Params &p, uint32_t tbase, i
           hv[i].y += v.y;
           hv[i].z += v.z;
           hv[i].w += v.w;
-          reinterpret_cast<float4 *>(out + dst[i] * p.N + tn * BN + c * 32)[lane & 7] = hv[i];
+          reinterpret_cast<float4 *>(out + dst[i] * p.N + col0 + c * 32)[lane & 7] = hv[i];
         }
       __syncwarp();
     }
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int64_t row = static_cast<int64_t>(tm) * BM + row_in_tile;
       const bool live = row < p.M;
       const uint32_t tbase = tmem_addr(tmem_base, quad * 32, acc * BN);
-      epilogue_rows<EPI>(p, tbase, row, live, tn, stg);
+      epilogue_rows<EPI>(p, tbase, row, live, EPI == SPTS_EPI_SWIGLU ? tn * 128 : tn * BN, BN, stg);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
@@ -349,6 +351,9 @@ spts_status launch_epi(const GemmArgs &g, const CUtensorMap &ta, const CUtensorM
 //               multicast to both CTAs);
 //   warps 2..5  epilogue of this CTA's rows; they release an accumulator on
 //               CTA 0's tempty[] barrier (128 arrivals from each CTA).
+// When the last round of tiles would keep at most half of the pairs busy,
+// those tiles run as two 128-column halves each (N = 128 MMAs, each CTA
+// supplying 64 rows of B), so the round takes half as long.
 // Loads are plain tile loads (no multicast): each CTA reads only its own
 // operand halves.  On exit the two CTAs reconcile the copies each issued per
 // stage so that CTA 0 can wait for every copy still in flight (a timeout may
@@ -367,6 +372,20 @@ __device__ __forceinline__ void tile_coords2(int t, int tiles_m2, int tiles_n, i
   const int r = t - grp * per_group;
   tm = first_m + r % gm;
   tn = r / gm;
+}
+
+// Unit u of a CTA pair's schedule: a whole 256-column tile, or, from tile
+// split_from on (the last round of tiles when it fills at most half of the
+// pairs), one of its two 128-column halves (half = 0 or 1; -1: whole tile).
+__device__ __forceinline__ void unit_coords2(int u, int split_from, int tiles_m2, int tiles_n, int &tm, int &tn,
+                                             int &half) {
+  int t = u;
+  half = -1;
+  if (u >= split_from) {
+    t = split_from + ((u - split_from) >> 1);
+    half = (u - split_from) & 1;
+  }
+  tile_coords2(t, tiles_m2, tiles_n, tm, tn);
 }
 
 template <int EPI>
@@ -411,6 +430,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem_base = *tmem_holder;
   const int tiles_m2 = (p.tiles_m + 1) >> 1;
   const int tiles = tiles_m2 * p.tiles_n;
+  const int units = p.split_from + 2 * (tiles - p.split_from);
   const int kblocks = p.K / BK;
 
   if (warp == 0) {
@@ -421,11 +441,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       const CUtensorMap *mb = (EPI == SPTS_EPI_SWIGLU && rank == 1) ? &tmB2 : &tmB;
       int stage = 0;
       uint32_t phase = 0;
-      for (int t = pair; t < tiles && !*abort_flag; t += n_pairs) {
-        int tm, tn;
-        tile_coords2(t, tiles_m2, p.tiles_n, tm, tn);
+      for (int t = pair; t < units && !*abort_flag; t += n_pairs) {
+        int tm, tn, half;
+        unit_coords2(t, p.split_from, tiles_m2, p.tiles_n, tm, tn, half);
         const int a_row = tm * 256 + static_cast<int>(rank) * 128;
-        const int b_row = EPI == SPTS_EPI_SWIGLU ? tn * 128 : tn * BN + static_cast<int>(rank) * 128;
+        // each CTA supplies half of the tile's N rows of B (a half tile: 64
+        // of the 128 rows its box loads; the rest is not read)
+        const int b_row = EPI == SPTS_EPI_SWIGLU ? tn * 128 + (half < 0 ? 0 : half * 64)
+                          : half < 0               ? tn * BN + static_cast<int>(rank) * 128
+                                                   : tn * BN + half * 128 + static_cast<int>(rank) * 64;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, p.wait_ns, 0x31u)) break;
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE2_BYTES);
@@ -442,12 +466,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (rank == 0) {  // the whole warp runs the issue loop; one elected lane issues each MMA and commit
-      constexpr uint32_t idesc = idesc_bf16_f32(256, BN, 0, 0);
+      constexpr uint32_t idesc_full = idesc_bf16_f32(256, BN, 0, 0);
+      constexpr uint32_t idesc_half = idesc_bf16_f32(256, BN / 2, 0, 0);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int t = pair; t < tiles && ok; t += n_pairs, ++local) {
+      for (int t = pair; t < units && ok; t += n_pairs, ++local) {
+        const uint32_t idesc = t < p.split_from ? idesc_full : idesc_half;
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!__all_sync(0xffffffffu,
@@ -484,18 +510,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int row_in_tile = quad * 32 + lane;
     float *stg = reinterpret_cast<float *>(smem + STAGES2 * STAGE2_BYTES + 256) + (warp - 2) * 32 * STG_STRIDE;
     int local = 0;
-    for (int t = pair; t < tiles; t += n_pairs, ++local) {
+    for (int t = pair; t < units; t += n_pairs, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, p.wait_ns, 0x34u);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      int tm, tn;
-      tile_coords2(t, tiles_m2, p.tiles_n, tm, tn);
+      int tm, tn, half;
+      unit_coords2(t, p.split_from, tiles_m2, p.tiles_n, tm, tn, half);
       const int64_t row = static_cast<int64_t>(tm) * 256 + rank * 128 + row_in_tile;
       const bool live = row < p.M;
       const uint32_t tbase = tmem_addr(tmem_base, quad * 32, acc * BN);
-      epilogue_rows<EPI>(p, tbase, row, live, tn, stg);
+      const int width = half < 0 ? BN : BN / 2;
+      const int col0 = EPI == SPTS_EPI_SWIGLU ? tn * 128 + (half < 0 ? 0 : half * 64)
+                                              : tn * BN + (half < 0 ? 0 : half * 128);
+      epilogue_rows<EPI>(p, tbase, row, live, col0, width, stg);
       tc_fence_before();
       mbar_arrive_remote(&tempty[acc], 0);
     }
@@ -556,7 +585,12 @@ spts_status launch_epi2(const CUtensorMap &ta, const CUtensorMap &tb, const CUte
     max_pairs = n > 0 ? n : 1;
   }
   const int tiles = ((p.tiles_m + 1) >> 1) * p.tiles_n;
-  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  // The last round of tiles, when it would keep at most half of the pairs
+  // busy, runs as 128-column halves: one round of half the length.
+  const int tail = tiles % max_pairs;
+  p.split_from = (tail > 0 && 2 * tail <= max_pairs) ? tiles - tail : tiles;
+  const int units = p.split_from + 2 * (tiles - p.split_from);
+  const int pairs = units < max_pairs ? units : max_pairs;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   SPTS_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm2_bf16_kernel<EPI>, ta, tb, tb2, p));
   note_launch();
