@@ -67,3 +67,20 @@ def test_importing_the_binding_loads_no_oracle_module():
             "raise SystemExit(1 if bad else 0)\n") % ROOT
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout + r.stderr
+
+
+def test_binding_without_the_library_fails_loudly(tmp_path):
+    # the package copied without libspts.so: importing it raises, it does not
+    # fall back to anything
+    import shutil
+    pkg = os.path.join(ROOT, "token_skipping_sparse_b200")
+    dst = tmp_path / "token_skipping_sparse_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "__pycache__", "csrc"))
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "try:\n"
+            "    import token_skipping_sparse_b200\n"
+            "except ImportError as e:\n"
+            "    print('RAISED', e); raise SystemExit(0)\n"
+            "raise SystemExit(1)\n") % str(tmp_path)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "no CPU fallback" in r.stdout, r.stdout + r.stderr
