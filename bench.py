@@ -762,6 +762,12 @@ def attention_arm(args, rank, world, dev):
                          "frac": round(ach / peaks["bf16"], 4), "traffic": None}}
 
 
+# Free candidates above which spts_select_topk runs on the grid (given a
+# workspace); the library's own threshold, checked against its source in the
+# host tests.
+TOPK_GRID_MIN = 20480
+
+
 def topk_arm(args, rank, world, dev):
     """spts_select_topk alone on a workload's candidate count: the FFN-set
     selection of the layer (MaxNorm-Add fusion of two seeded positive score
@@ -799,7 +805,7 @@ def topk_arm(args, rank, world, dev):
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded exponential and |N(26, 2)| score vectors)",
             "config": {"workload": wl.name, "kernel": "select_topk", "Nc": N, "k": k, "force_tail": wl.P,
-                       "fuse": "maxnorm_add", "path": "grid" if N - wl.P > 20480 else "one CTA"},
+                       "fuse": "maxnorm_add", "path": "grid" if N - wl.P > TOPK_GRID_MIN else "one CTA"},
             "roofline": {"bound": "latency", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 5), "traffic": None,
                          "note": f"{nbytes / 1e6:.2f} MB per call: far below what HBM time would matter for; the "

@@ -97,3 +97,10 @@ def test_cpu_baseline_times_one_whole_layer():
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
     assert abs(cb["value"] * cb["seconds"] - wl.N) <= 0.05 * wl.N   # seconds is rounded to 1 ms
     assert "unavailable" in bench.cpu_baseline(WORKLOADS["layer_small_kv"])
+
+
+def test_topk_path_label_matches_the_library_threshold():
+    import re
+    src = open(os.path.join(bench.ROOT, "token_skipping_sparse_b200", "csrc", "topk.cu")).read()
+    m = re.search(r"#define TK_GRID_MIN (\d+)", src)
+    assert m and int(m.group(1)) == bench.TOPK_GRID_MIN
